@@ -1,0 +1,32 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a CUDA B200 (sm_100a) and the built library")
+    config.addinivalue_line(
+        "markers", "slow: full-size workload checks (minutes)")
+
+
+def pytest_collection_modifyitems(config, items):
+    # GPU tests must never run silently on a machine without a GPU: skip them
+    # there (the CPU suite is run with -m "not gpu" anyway), but on a machine
+    # with a GPU they run and must find the native library.
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:
+        has_gpu = False
+    if has_gpu:
+        return
+    skip = pytest.mark.skip(reason="no CUDA device on this host")
+    for item in items:
+        if "gpu" in item.keywords:
+            item.add_marker(skip)

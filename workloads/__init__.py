@@ -1,0 +1,137 @@
+"""Seeded synthetic inputs for the attention workloads.
+
+This module only draws random numbers and rounds them to the storage dtype.
+It holds none of the attention arithmetic, so both the fp64 CPU oracle and
+the CUDA path can take their inputs from here without sharing any of the
+method's code.
+
+Workloads (shapes are [B, H, N, d], d fastest):
+
+* ``fp32_small``  B1 H2 N256 d64, fp32, forward only, non-causal.
+* ``fwd_d64``     B8 H16 N1024 d64, bf16, forward only, non-causal.
+* ``causal_d128`` B4 H16 N4096 d128, bf16, causal, forward+backward.
+* ``long_d128``   B1 H16 N16384 d128, bf16, causal, forward+backward.
+* ``gpt3_d80``    B8 H32 N2048 d80, bf16, causal, forward+backward; Q, K, V
+  are projections X.W of a unit-normal activation X [B, N, 2560] through
+  three independent N(0, 0.02^2) [2560, 2560] weights, then split into
+  32 heads of 80 (the GPT-3 2.7B layer shape named on the FlashAttention-2
+  review page, section on results, GPT-3 2.7B end-to-end training).
+
+Every tensor is generated in fp32 on the CPU from ``torch.Generator`` seeded
+with ``1000 + index`` and then rounded (round-to-nearest-even) to the storage
+dtype, so the GPU and the oracle see the same bits.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    index: int
+    B: int
+    H: int
+    N: int
+    d: int
+    dtype: str          # "fp32" or "bf16"
+    causal: bool
+    backward: bool
+    projected: bool = False   # Q/K/V = X.W (GPT-3 shaped layer)
+    hidden: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def seed(self) -> int:
+        return 1000 + self.index
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "fp32" else torch.bfloat16
+
+    def describe(self) -> str:
+        pas = "fwd+bwd" if self.backward else "fwd"
+        cz = "causal" if self.causal else "non-causal"
+        return (f"{self.name}: B{self.B} H{self.H} N{self.N} d{self.d} "
+                f"{self.dtype} {cz} {pas}")
+
+
+WORKLOADS: Dict[str, Workload] = {
+    w.name: w for w in [
+        Workload("fp32_small", 0, 1, 2, 256, 64, "fp32", False, False),
+        Workload("fwd_d64", 1, 8, 16, 1024, 64, "bf16", False, False),
+        Workload("causal_d128", 2, 4, 16, 4096, 128, "bf16", True, True),
+        Workload("long_d128", 3, 1, 16, 16384, 128, "bf16", True, True),
+        Workload("gpt3_d80", 4, 8, 32, 2048, 80, "bf16", True, True,
+                 projected=True, hidden=2560),
+    ]
+}
+
+
+def round_to(x: torch.Tensor, dtype: torch.dtype) -> torch.Tensor:
+    """Round an fp32 tensor to ``dtype`` (RNE) and keep it in that dtype."""
+    return x.to(dtype).contiguous()
+
+
+def randn(shape, seed: int, dtype: torch.dtype = torch.bfloat16,
+          std: float = 1.0) -> torch.Tensor:
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    x = torch.randn(*shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        x = x * std
+    return round_to(x, dtype)
+
+
+def make_inputs(w: Workload, with_grad_out: Optional[bool] = None,
+                B: Optional[int] = None, H: Optional[int] = None,
+                N: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Seeded CPU inputs for workload ``w``.
+
+    B/H/N may be overridden to draw a smaller instance with the same
+    distribution (used by sampled and reduced-size checks).  Returns q, k,
+    v (and do when a backward is requested), contiguous [B, H, N, d].
+    """
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    N = w.N if N is None else N
+    want_do = w.backward if with_grad_out is None else with_grad_out
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    dt = w.torch_dtype
+    out: Dict[str, torch.Tensor] = {}
+    if w.projected:
+        hid = w.hidden
+        hid_eff = H * w.d
+        x = torch.randn(B, N, hid, generator=g, dtype=torch.float32)
+        for name in ("q", "k", "v"):
+            wmat = torch.randn(hid, hid_eff, generator=g, dtype=torch.float32) * 0.02
+            proj = torch.matmul(x, wmat)                      # [B, N, H*d] fp32
+            proj = proj.view(B, N, H, w.d).permute(0, 2, 1, 3).contiguous()
+            out[name] = round_to(proj, dt)
+    else:
+        for name in ("q", "k", "v"):
+            out[name] = round_to(
+                torch.randn(B, H, N, w.d, generator=g, dtype=torch.float32), dt)
+    if want_do:
+        out["do"] = round_to(
+            torch.randn(B, H, N, w.d, generator=g, dtype=torch.float32), dt)
+    return out
+
+
+def random_case(B: int, H: int, N: int, d: int, seed: int,
+                dtype: torch.dtype = torch.bfloat16, grad: bool = True,
+                std: float = 1.0) -> Dict[str, torch.Tensor]:
+    """Small seeded iid-normal case (parity tests at odd sizes)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    out = {}
+    names = ("q", "k", "v", "do") if grad else ("q", "k", "v")
+    for name in names:
+        x = torch.randn(B, H, N, d, generator=g, dtype=torch.float32) * std
+        out[name] = round_to(x, dtype)
+    return out
