@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark: exact attention forward+backward TFLOP/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-cpu-baseline] [--sweep]
+
+One step is one pass of the whole hot path over one batch: the forward
+(fa_forward: O and LSE) followed by the backward (fa_backward: D
+preprocess, the dK/dV/dQ kernel, the dQ conversion) of the workload, inputs
+resident in HBM.  Throughput counts the algorithmic FLOPs of both passes
+(forward 4 B H N^2 d, halved when causal; backward 2.5x the forward).
+
+Default workload: causal_d128 (B4 H16 N4096 d128, bf16, causal fwd+bwd),
+the configuration the metric's target is stated at (N >= 4096, d = 128).
+Its working set (~0.7 GB) is larger than the 126 MB L2, so no flush is needed
+between steps.  Under torchrun each rank runs the same per-GPU workload on its
+own GPU (independent heads, no collective on the data path: weak scaling);
+the time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this
+project has) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+from exact_io_aware_99_b200 import perf  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOPs/s (bf16, 1 B200) and % of dense tensor peak vs N"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.proc is None:
+            return out
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        except Exception:
+            return out
+        if not rows:
+            return out
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        out.update(sm_mhz=statistics.median(sm) if sm else None,
+                   sm_max_mhz=max(mx) if mx else None, reasons=sorted(reasons),
+                   samples=len(rows))
+        return out
+
+
+# --------------------------------------------------------------- ncu traffic
+
+KERNEL_SOURCES = {
+    "bwd": ["exact_io_aware_99_b200/csrc/fa_bwd_sm100.cu", "exact_io_aware_99_b200/csrc/sm100.cuh"],
+    "fwd": ["exact_io_aware_99_b200/csrc/fa_fwd_sm100.cu", "exact_io_aware_99_b200/csrc/sm100.cuh"],
+}
+
+
+def source_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_ncu.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source_sha256:\s*([0-9a-f]+)", text)
+    if not m or m.group(2) != source_hash(kernel):
+        return None
+    return float(m.group(1))
+
+
+# --------------------------------------------------------------- our impl
+
+def run_ours(args, peaks, peak_kind):
+    import exact_io_aware_99_b200 as fa
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = workloads.WORKLOADS[args.workload]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    x = workloads.make_inputs(w, with_grad_out=True)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wbytes = fa.fa_backward_workspace_size(B, H, N, d)
+    wsbuf = torch.empty(wbytes, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    scale, causal = w.scale, w.causal
+
+    def fwd():
+        fa.fa_forward(q, k, v, o, lse, B, H, N, d, scale, causal, sp)
+
+    def bwd():
+        fa.fa_backward(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, causal, wsbuf, wbytes,
+                       sp)
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    st, site = fa.fa_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError(f"device wait timed out in warm-up (site {site:#x})")
+
+    # Device-timed region: K steps, events on the launching stream around
+    # each pass so the per-pass (kernel) durations are measured live.
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler start
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        fwd()
+        ev[i][1].record(stream)
+        bwd()
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    bwd_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    st, site = fa.fa_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError(f"device wait timed out (site {site:#x})")
+    if ws > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+
+    flops_f = perf.fwd_flops(B, H, N, d, causal)
+    flops_b = perf.bwd_flops(B, H, N, d, causal)
+    step_flops = flops_f + flops_b
+    value = ws * step_flops / (ms_step * 1e-3) / 1e12
+
+    # End to end through the public API with host buffers: pinned host inputs
+    # copied in, both passes, outputs copied back, every step.
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (x[n].pin_memory() for n in ("q", "k", "v", "do"))
+        ho, hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(4))
+        hlse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+        bi = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        bo = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            do.copy_(hdo, non_blocking=True)
+            fwd()
+            bwd()
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ne = max(3, min(args.steps, 10))
+        a.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = a.elapsed_time(b) / ne
+        if ws > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": round(ws * step_flops / (e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e_ms, 4)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peak = float(peaks["bf16_tflops"])
+    peak_s = float(peaks.get("bf16_tflops_sustained", peak))
+    bwd_tf = flops_b / (bwd_ms * 1e-3) / 1e12
+    fwd_tf = flops_f / (fwd_ms * 1e-3) / 1e12
+    traffic = recorded_traffic("bwd", args.workload)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded iid N(0,1), rounded to bf16)",
+        "config": {"workload": w.describe(), "B": B, "H": H, "N": N, "d": d,
+                   "causal": causal, "passes": "fwd+bwd",
+                   "l2": "working set ~%.2f GB > 126 MB L2 (no flush needed)"
+                         % ((7 * B * H * N * d * 2 + wbytes) / 1e9),
+                   "parallelism": f"{ws} independent replicas" if ws > 1 else "single GPU"},
+        "fwd_tflops": round(fwd_tf, 3), "bwd_tflops": round(bwd_tf, 3),
+        "fwd_frac_of_peak": round(fwd_tf / peak, 4), "bwd_frac_of_peak": round(bwd_tf / peak, 4),
+        "frac_of_peak": round(value / ws / peak, 4),
+        "frac_of_sustained_peak": round(value / ws / peak_s, 4),
+        "peak_source": f"{peak_kind} (MEASURED_PEAKS.json bf16_tflops burst {peak}, "
+                       f"sustained {peak_s})",
+        "roofline": {"kernel": "fa_backward (preprocess + dK/dV/dQ kernel + dQ convert)",
+                     "bound": "tensor", "achieved": round(bwd_tf, 3), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(bwd_tf / peak, 4),
+                     "traffic": traffic,
+                     "algorithmic_bytes": perf.bwd_bytes(B, H, N, d)},
+        "gpu_launches": 4 * args.steps,
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                   "reasons": clk["reasons"], "samples": clk["samples"]},
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    return line
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(w, seconds: float):
+    """The fp64 oracle (as it stands) on a bounded sample of the workload:
+    whole heads, forward and backward, until about ``seconds`` of CPU work."""
+    import oracle
+    x = workloads.make_inputs(w, with_grad_out=True, B=1)
+    cores = os.cpu_count() or 1
+    n_heads, flops, t0 = 0, 0.0, time.perf_counter()
+    per_head = perf.fwd_flops(1, 1, w.N, w.d, w.causal) + perf.bwd_flops(1, 1, w.N, w.d, w.causal)
+    while True:
+        h = n_heads % w.H
+        qh, kh, vh, doh = (x[n][0, h] for n in ("q", "k", "v", "do"))
+        oracle.attention_forward(qh, kh, vh, w.scale, w.causal)
+        oracle.attention_backward(qh, kh, vh, doh, w.scale, w.causal)
+        n_heads += 1
+        flops += per_head
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    return {"value": round(flops / el / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_heads} head(s) of {w.name} (N={w.N}, d={w.d}), fwd+bwd, fp64 numpy "
+                      f"on the host ({el:.1f} s)"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    w = workloads.WORKLOADS[args.workload]
+    x = workloads.make_inputs(w, with_grad_out=True, B=1)
+    per_head = perf.fwd_flops(1, 1, w.N, w.d, w.causal) + perf.bwd_flops(1, 1, w.N, w.d, w.causal)
+
+    def step(i):
+        h = i % w.H
+        qh, kh, vh, doh = (x[n][0, h] for n in ("q", "k", "v", "do"))
+        oracle.attention_forward(qh, kh, vh, w.scale, w.causal)
+        oracle.attention_backward(qh, kh, vh, doh, w.scale, w.causal)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    value = per_head * args.steps / el / 1e12
+    cores = os.cpu_count() or 1
+    sample = f"1 head of {w.name} (N={w.N}, d={w.d}) fwd+bwd per step, fp64 numpy oracle"
+    return {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.describe(), "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "causal": w.causal, "passes": "fwd+bwd"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def run_sweep(args, peaks):
+    """Forward and backward TFLOP/s vs N at d = 128, causal and not, holding
+    B*H*N = 262144 (one line per point; not the benchmark line)."""
+    import exact_io_aware_99_b200 as fa
+    peak = float(peaks["bf16_tflops"])
+    for causal in (True, False):
+        for N in (512, 1024, 2048, 4096, 8192, 16384):
+            d = 128
+            H = 16
+            B = max(1, 262144 // (H * N))
+            x = workloads.random_case(B, H, N, d, N, grad=True)
+            q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+            o = torch.empty_like(q)
+            lse = torch.empty((B, H, N), device="cuda")
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+            wb = fa.fa_backward_workspace_size(B, H, N, d)
+            wsb = torch.empty(wb, device="cuda", dtype=torch.uint8)
+            sc = 1 / math.sqrt(d)
+
+            def f():
+                fa.fa_forward(q, k, v, o, lse, B, H, N, d, sc, causal)
+
+            def g():
+                fa.fa_backward(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, sc, causal, wsb, wb)
+
+            res = {}
+            for name, fn, fl in (("fwd", f, perf.fwd_flops(B, H, N, d, causal)),
+                                 ("bwd", g, perf.bwd_flops(B, H, N, d, causal))):
+                for _ in range(3):
+                    f()
+                    fn()
+                torch.cuda.synchronize()
+                a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+                n = 10
+                a.record()
+                for _ in range(n):
+                    fn()
+                b.record()
+                torch.cuda.synchronize()
+                ms = a.elapsed_time(b) / n
+                res[name] = fl / (ms * 1e-3) / 1e12
+            print(json.dumps({"sweep": "d128", "causal": causal, "B": B, "H": H, "N": N,
+                              "fwd_tflops": round(res["fwd"], 2),
+                              "bwd_tflops": round(res["bwd"], 2),
+                              "fwd_frac": round(res["fwd"] / peak, 4),
+                              "bwd_frac": round(res["bwd"] / peak, 4)}), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description="exact attention fwd+bwd benchmark (B200)")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="causal_d128", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--sweep", action="store_true", help="print the TFLOP/s-vs-N sweep instead")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    peaks, kind = load_peaks()
+    if args.impl == "reference":
+        line = run_reference(args)
+    elif args.sweep:
+        run_sweep(args, peaks)
+        return
+    else:
+        line = run_ours(args, peaks, kind)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,291 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument checks, TMA
+// tensor-map encoding, workspace carving and kernel launches.  No device
+// memory is allocated here; the only device state is the status word below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace {
+
+// Written by a kernel whose bounded wait ran out (first site wins).
+__device__ int g_fa_status = 0;
+
+constexpr unsigned long long kDefaultLimitNs = 2000000000ull;
+std::atomic<unsigned long long> g_limit_ns{kDefaultLimitNs};
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  int checked = 0;  // 0 unknown, 1 supported, -1 unsupported
+  int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+fa_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_CUDA;
+}
+
+// Checks that the current device is an sm_100 part and returns its launch
+// context (status-word address, time limit).
+fa_status device_context(void* stream, fa::Launch* L) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  DeviceInfo& di = g_dev[dev];
+  if (di.checked == 0) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (di.checked == 0) {
+      cudaDeviceProp prop;
+      e = cudaGetDeviceProperties(&prop, dev);
+      if (e != cudaSuccess) return cuda_fail(e);
+      if (prop.major != 10 || prop.minor != 0) {
+        di.checked = -1;
+      } else {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_fa_status);
+        if (e != cudaSuccess) return cuda_fail(e);
+        di.status = static_cast<int*>(p);
+        di.checked = 1;
+      }
+    }
+  }
+  if (di.checked < 0) return FA_ERR_UNSUPPORTED;
+  L->stream = static_cast<cudaStream_t>(stream);
+  L->status = di.status;
+  L->limit_ns = g_limit_ns.load(std::memory_order_relaxed);
+  return FA_OK;
+}
+
+fa_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode ? FA_OK : FA_ERR_CUDA;
+}
+
+// [BH, N, d] bf16 viewed as 3-D {d, N, BH}; box {64, 128, 1}; 128-byte
+// swizzle; out-of-range rows and columns read as zero.
+fa_status make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = static_cast<int>(r);
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_common(int B, int H, int N, int d, float scale, fa_dtype dtype) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (dtype == FA_BF16) {
+    if (d != 64 && d != 80 && d != 128) return FA_ERR_UNSUPPORTED;
+    if ((N + 127) / 128 > 65535) return FA_ERR_UNSUPPORTED;  // grid.y limit
+    if (static_cast<long long>(N) * d * 2 * bh >= (1LL << 40)) return FA_ERR_UNSUPPORTED;
+  } else if (dtype == FA_FP32) {
+    if (d < 1 || d > 128) return FA_ERR_UNSUPPORTED;
+    if ((N + 63) / 64 > 65535) return FA_ERR_UNSUPPORTED;
+  } else {
+    return FA_ERR_UNSUPPORTED;
+  }
+  return FA_OK;
+}
+
+struct WsLayout {
+  size_t dq_off, dvec_off, lse2_off, total;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+WsLayout ws_layout(int B, int H, int N, int d) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t np = static_cast<size_t>(fa::round_up(N, fa::kTileRows));
+  WsLayout w;
+  w.dq_off = 0;
+  w.dvec_off = up256(bh * N * d * sizeof(float));
+  w.lse2_off = w.dvec_off + up256(bh * np * sizeof(float));
+  w.total = w.lse2_off + up256(bh * np * sizeof(float));
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case FA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case FA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case FA_ERR_CUDA: return "CUDA call failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+int fa_last_cuda_error(void) { return g_last_cuda_error; }
+
+void fa_set_wait_timeout_ns(unsigned long long ns) {
+  g_limit_ns.store(ns ? ns : kDefaultLimitNs, std::memory_order_relaxed);
+}
+
+fa_status fa_device_status(int reset, int* site) {
+  fa::Launch L;
+  fa_status st = device_context(nullptr, &L);
+  if (st != FA_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_fa_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (reset && v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (site) *site = v;
+  return v ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+}
+
+fa_status fa_selftest_wait_timeout(void* stream) {
+  fa::Launch L;
+  fa_status st = device_context(stream, &L);
+  if (st != FA_OK) return st;
+  cudaError_t e = fa::launch_selftest_wait(L);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+fa_status fa_forward_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int N, int d, float scale, int causal, fa_dtype dtype,
+                        void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_MISALIGNED;
+  fa::Launch L;
+  st = device_context(stream, &L);
+  if (st != FA_OK) return st;
+  const int BH = B * H;
+  const int cz = causal ? 1 : 0;
+  cudaError_t e;
+  if (dtype == FA_FP32) {
+    e = fa::launch_fwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                           static_cast<const float*>(v), static_cast<float*>(o), lse, BH, N, d,
+                           scale, cz, L);
+  } else {
+    st = get_encoder();
+    if (st != FA_OK) return st;
+    CUtensorMap tq, tk, tv;
+    if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
+    if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
+    if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
+    e = fa::launch_fwd_sm100(tq, tk, tv, o, lse, BH, N, d, scale, cz, L);
+  }
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int N, int d, float scale, int causal, void* stream) {
+  return fa_forward_ex(q, k, v, o, lse, B, H, N, d, scale, causal, FA_BF16, stream);
+}
+
+size_t fa_backward_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || d > 128) return 0;
+  return ws_layout(B, H, N, d).total;
+}
+
+fa_status fa_backward_ex(const void* q, const void* k, const void* v, const void* o,
+                         const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, float scale, int causal, void* workspace,
+                         size_t workspace_bytes, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  const WsLayout w = ws_layout(B, H, N, d);
+  if (!workspace || workspace_bytes < w.total ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FA_ERR_WORKSPACE;
+  fa::Launch L;
+  st = device_context(stream, &L);
+  if (st != FA_OK) return st;
+  const int BH = B * H;
+  const int cz = causal ? 1 : 0;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws + w.dq_off);
+  float* dvec = reinterpret_cast<float*>(ws + w.dvec_off);
+  float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
+  cudaError_t e;
+  if (dtype == FA_FP32) {
+    e = fa::launch_bwd_preprocess(o, dO, lse, dvec, nullptr, nullptr, BH, N, d, 0, L);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = fa::launch_bwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                           static_cast<const float*>(v), static_cast<const float*>(dO), lse, dvec,
+                           static_cast<float*>(dq), static_cast<float*>(dk),
+                           static_cast<float*>(dv), BH, N, d, scale, cz, L);
+    return e == cudaSuccess ? FA_OK : cuda_fail(e);
+  }
+  st = get_encoder();
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&tdo, dO, BH, N, d)) != FA_OK) return st;
+  e = fa::launch_bwd_preprocess(o, dO, lse, dvec, lse2, dq_acc, BH, N, d, 1, L);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, dvec, lse2, dq_acc, dk, dv, BH, N, d, scale, cz, L);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = fa::launch_dq_convert_bf16(dq_acc, dq, static_cast<size_t>(BH) * N * d, L);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+fa_status fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                      float scale, int causal, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  return fa_backward_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+                        workspace_bytes, FA_BF16, stream);
+}
+
+}  // extern "C"

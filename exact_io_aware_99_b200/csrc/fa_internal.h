@@ -1,0 +1,68 @@
+// fa_internal.h -- launch interface between the C ABI (fa_api.cu) and the
+// kernel translation units.  Not installed; not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+struct Launch {
+  cudaStream_t stream;
+  int* status;                  // device status word
+  unsigned long long limit_ns;  // bounded-wait time limit
+};
+
+// Wait-site codes recorded in the status word when a bounded wait runs out.
+enum WaitSite : int {
+  kSiteFwdProducer = 0x101,
+  kSiteFwdMma = 0x102,
+  kSiteFwdSoftmax = 0x103,
+  kSiteFwdEpilogue = 0x104,
+  kSiteFwdDrain = 0x105,
+  kSiteBwdProducer = 0x201,
+  kSiteBwdMma = 0x202,
+  kSiteBwdSoftmax = 0x203,
+  kSiteBwdDq = 0x204,
+  kSiteBwdEpilogue = 0x205,
+  kSiteBwdDrain = 0x206,
+  kSiteSelfTest = 0x7e57,
+};
+
+// Rows of a head are padded to a multiple of this in the backward's row
+// vectors (D and the base-2 LSE), and it is the tile height of every kernel.
+constexpr int kTileRows = 128;
+
+inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// --- bf16 tensor-core path (fa_fwd_sm100.cu, fa_bwd_sm100.cu) -------------
+// Tensor maps describe a [BH, N, d] bf16 tensor as 3-D {d, N, BH} with a
+// {64, 128, 1} box and 128-byte swizzle.
+cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             void* o, float* lse, int BH, int N, int d, float scale, int causal,
+                             const Launch& L);
+
+cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tdo, const float* dvec, const float* lse2,
+                             float* dq_acc, void* dk, void* dv, int BH, int N, int d, float scale,
+                             int causal, const Launch& L);
+
+// --- helpers shared by both dtypes (fa_simt.cu) ---------------------------
+// D = rowsum(dO o O) (fp32, padded rows = 0), lse2 = LSE * log2(e) (padded
+// rows = +inf), and zero the fp32 dQ accumulator.
+cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse, float* dvec,
+                                  float* lse2, float* dq_acc, int BH, int N, int d, int is_bf16,
+                                  const Launch& L);
+cudaError_t launch_dq_convert_bf16(const float* dq_acc, void* dq, size_t n, const Launch& L);
+
+// --- fp32 SIMT path (fa_simt.cu) -------------------------------------------
+cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                           int BH, int N, int d, float scale, int causal, const Launch& L);
+cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const float* dO,
+                           const float* lse, const float* dvec, float* dq, float* dk, float* dv,
+                           int BH, int N, int d, float scale, int causal, const Launch& L);
+
+cudaError_t launch_selftest_wait(const Launch& L);
+
+}  // namespace fa

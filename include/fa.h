@@ -1,0 +1,179 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa_sm100.so).
+ *
+ * The library computes exact scaled-dot-product attention and its gradient
+ * without ever writing the N x N score or probability matrices to device
+ * memory:
+ *
+ *   forward   O = softmax(scale * Q K^T [+ causal mask]) V,
+ *             LSE_i = m_i + ln(l_i)   (m: row max of the scaled scores,
+ *                                      l: row sum of exp(score - m))
+ *   backward  dV = P^T dO, dP = dO V^T, dS = P o (dP - rowsum(dO o O)),
+ *             dQ = scale dS K, dK = scale dS^T Q, with P recomputed from Q, K
+ *             and the saved LSE.
+ *
+ * Passages that define the operations (web pages on FlashAttention):
+ *   - "FlashAttention-2: Faster Attention with Better Parallelism and Work
+ *     Partitioning" review page: core-algorithm answer, section 1 (S = QK^T,
+ *     P = softmax(S), O = PV), section 2 (1) tiling with B_r x B_c blocks,
+ *     (2) forward pass with a running max m and running sum l, (3) backward
+ *     pass recomputing softmax from the saved (m, l) and forming dQ, dK, dV;
+ *     the FLOP answer (forward 4 N^2 d, backward 2.5x forward; O(N) extra
+ *     memory for the softmax statistics).
+ *   - "IO-4 FlashAttention (Memory IO optimisation based attention
+ *     acceleration)" note: the scaled form softmax(QK^T / sqrt(d_k)) V;
+ *     section 4 online softmax; section 5 O(n) memory.
+ *   - "[LLM] Flash Attention" blog post: "Recomputation" (S, P recomputed
+ *     in the backward instead of stored).
+ * Readings where the pages are silent or garbled: the causal mask hides key
+ * j from query i when j > i; the saved statistic is the single natural-log
+ * LSE; the page's dS formula is read as the row-wise softmax Jacobian and
+ * the scale is applied to dQ and dK (chain rule through S = scale Q K^T).
+ *
+ * Conventions for every entry point
+ *   Layout     q, k, v, o, dO, dq, dk, dv: contiguous [B, H, N, d] row-major
+ *              (d fastest); lse: contiguous [B, H, N] fp32, natural log.
+ *   Pointers   device pointers, each 16-byte aligned; the caller owns all
+ *              memory.  The library never allocates device memory.  It keeps
+ *              one 4-byte device status word per process (a file-scope
+ *              device variable) and nothing else.
+ *   Streams    `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *              default stream).  Every call is asynchronous on that stream;
+ *              no call synchronises the host except fa_device_status.
+ *   Errors     argument errors are reported before anything is launched and
+ *              no output is touched; launch errors map to FA_ERR_CUDA.
+ *              Kernels never trap: a device-side wait that runs past its time
+ *              limit records the fact in the status word, the kernel returns,
+ *              and fa_device_status reports FA_ERR_DEVICE_TIMEOUT.
+ *   Outputs    are overwritten, never accumulated into.
+ *   Devices    sm_100a (B200) only; any other device gives FA_ERR_UNSUPPORTED.
+ */
+#ifndef FA_SM100_H_
+#define FA_SM100_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1,     /* null pointer, B/H/N < 1, non-finite or non-positive scale */
+  FA_ERR_UNSUPPORTED = -2,     /* head dim or dtype not built, or not an sm_100 device */
+  FA_ERR_MISALIGNED = -3,      /* a pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = -4,       /* workspace null, too small or not 256-byte aligned */
+  FA_ERR_CUDA = -5,            /* a CUDA runtime/driver call failed (see fa_last_cuda_error) */
+  FA_ERR_DEVICE_TIMEOUT = -6   /* a kernel's bounded wait ran out (reported by fa_device_status) */
+} fa_status;
+
+typedef enum {
+  FA_BF16 = 0,   /* bf16 storage, fp32 accumulation on the tensor cores */
+  FA_FP32 = 1    /* fp32 storage and fp32 FMA arithmetic (small-case path) */
+} fa_dtype;
+
+/*
+ * fa_forward -- bf16 forward.
+ *   q, k, v  [B, H, N, d] bf16 inputs.
+ *   o        [B, H, N, d] bf16 output (the normalised attention output).
+ *   lse      [B, H, N] fp32 output, LSE_i = ln sum_j exp(scale q_i.k_j) over
+ *            the keys query i sees.
+ *   d        head dimension: 64, 80 or 128.
+ *   N        sequence length, any N >= 1 (ragged tails are masked).
+ *   scale    score multiplier (1/sqrt(d) for standard attention), > 0.
+ *   causal   0: every query sees every key; 1: query i sees keys j <= i.
+ */
+FA_API fa_status fa_forward(const void* q, const void* k, const void* v, void* o,
+                     float* lse, int B, int H, int N, int d, float scale,
+                     int causal, void* stream);
+
+/*
+ * fa_forward_ex -- as fa_forward with an explicit storage dtype.
+ *   FA_BF16: identical to fa_forward.
+ *   FA_FP32: q, k, v, o are fp32; any d in [1, 128]; fp32 arithmetic
+ *            throughout (no tensor-core rounding), for accuracy checks.
+ */
+FA_API fa_status fa_forward_ex(const void* q, const void* k, const void* v, void* o,
+                        float* lse, int B, int H, int N, int d, float scale,
+                        int causal, fa_dtype dtype, void* stream);
+
+/*
+ * fa_backward_workspace_size -- bytes of device scratch fa_backward needs:
+ * an fp32 dQ accumulator [B, H, N, d] plus two fp32 row vectors per head
+ * padded to a multiple of 128 rows (D = rowsum(dO o O) and the base-2 LSE),
+ * each part rounded up to 256 bytes.  Linear in N (no N x N buffer).
+ * Returns 0 for arguments that fa_backward would reject.
+ */
+FA_API size_t fa_backward_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_backward -- bf16 backward.
+ *   q, k, v, o, dO  [B, H, N, d] bf16 inputs (o is the forward output).
+ *   lse             [B, H, N] fp32, the forward's LSE.
+ *   dq, dk, dv      [B, H, N, d] bf16 outputs.
+ *   workspace       device scratch of at least
+ *                   fa_backward_workspace_size(B, H, N, d) bytes, 256-byte
+ *                   aligned, owned by the caller; its contents on entry do
+ *                   not matter and are clobbered.  Two calls that overlap on
+ *                   the GPU must not share one workspace.
+ *   Other arguments as in fa_forward (same scale and causal as the forward).
+ * Launches three kernels in stream order (preprocess, main, dQ convert).
+ */
+FA_API fa_status fa_backward(const void* q, const void* k, const void* v,
+                      const void* o, const void* dO, const float* lse,
+                      void* dq, void* dk, void* dv,
+                      int B, int H, int N, int d, float scale, int causal,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_backward_ex -- as fa_backward with an explicit storage dtype.
+ *   FA_FP32: all tensors fp32, any d in [1, 128], fp32 arithmetic.
+ */
+FA_API fa_status fa_backward_ex(const void* q, const void* k, const void* v,
+                         const void* o, const void* dO, const float* lse,
+                         void* dq, void* dk, void* dv,
+                         int B, int H, int N, int d, float scale, int causal,
+                         void* workspace, size_t workspace_bytes,
+                         fa_dtype dtype, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FA_API const char* fa_status_string(fa_status s);
+
+/* The cudaError_t value of the last call that returned FA_ERR_CUDA on this
+ * host thread (0 if none). */
+FA_API int fa_last_cuda_error(void);
+
+/*
+ * fa_device_status -- synchronise the current device, then report whether a
+ * kernel of this library recorded a wait timeout since the last reset.
+ * Returns FA_OK or FA_ERR_DEVICE_TIMEOUT; *site (if non-NULL) receives the
+ * recorded wait-site code (0 when none).  reset != 0 clears the word.
+ */
+FA_API fa_status fa_device_status(int reset, int* site);
+
+/*
+ * fa_set_wait_timeout_ns -- time limit of every device-side wait in kernels
+ * launched after this call (default 2e9 ns).  0 restores the default.
+ */
+FA_API void fa_set_wait_timeout_ns(unsigned long long ns);
+
+/*
+ * fa_selftest_wait_timeout -- failure-detection self test: launches one
+ * 32-thread block that waits on a barrier nothing ever completes, under the
+ * current time limit; the wait gives up, records its site code (0x7e57) in
+ * the status word and the kernel returns.  The caller then reads
+ * fa_device_status.  Nothing faults, traps or hangs.
+ */
+FA_API fa_status fa_selftest_wait_timeout(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* FA_SM100_H_ */

@@ -1,0 +1,140 @@
+"""Host-side checks that need no GPU: the C-ABI library loads and exports
+every entry point the header declares, argument errors are reported before
+anything touches a device, the workspace formula is linear in N, and the
+benchmark's FLOP counter reproduces the page's worked numbers."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import workloads
+from exact_io_aware_99_b200 import perf
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def _lib():
+    import exact_io_aware_99_b200 as fa
+    return fa
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("fa_forward", "fa_backward", "fa_backward_workspace_size", "fa_status_string"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    fa = _lib()
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(declared_symbols()) == set(fa.EXPORTS)
+
+
+def test_status_strings():
+    fa = _lib()
+    assert fa.fa_status_string(0) == "ok"
+    for code in (-1, -2, -3, -4, -5, -6):
+        s = fa.fa_status_string(code)
+        assert s and s != "unknown status"
+    assert fa.fa_status_string(12345) == "unknown status"
+
+
+# Each of these must be rejected before any CUDA call (so they pass on a
+# machine without a GPU).  Pointers are fake but 256-byte aligned.
+A = 1 << 20
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(q=0), -1),                     # null pointer
+    (dict(B=0), -1), (dict(H=0), -1), (dict(N=0), -1),   # empty problem
+    (dict(scale=0.0), -1), (dict(scale=float("nan")), -1), (dict(scale=-1.0), -1),
+    (dict(d=96), -2), (dict(d=32), -2), (dict(d=256), -2),
+    (dict(q=A + 8), -3), (dict(o=A + 4), -3), (dict(lse=A + 2), -3),
+])
+def test_forward_argument_errors(args, code):
+    fa = _lib()
+    kw = dict(q=A, k=2 * A, v=3 * A, o=4 * A, lse=5 * A, B=1, H=2, N=256, d=64, scale=0.125)
+    kw.update(args)
+    st = fa.fa_forward(kw["q"], kw["k"], kw["v"], kw["o"], kw["lse"], kw["B"], kw["H"],
+                       kw["N"], kw["d"], kw["scale"], 0, stream=0, check=False)
+    assert st == code
+
+
+def test_fp32_path_accepts_any_small_head_dim_but_not_above_128():
+    fa = _lib()
+    st = fa.fa_forward_ex(A, 2 * A, 3 * A, 4 * A, 5 * A, 1, 1, 16, 129, 0.1, 0, fa.FA_FP32,
+                          stream=0, check=False)
+    assert st == fa.FA_ERR_UNSUPPORTED
+    st = fa.fa_forward_ex(A, 2 * A, 3 * A, 4 * A, 5 * A, 1, 1, 16, 7, 0.1, 0, 7,
+                          stream=0, check=False)
+    assert st == fa.FA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("ws_ptr,ws_bytes,code", [
+    (0, 1 << 30, -4),            # null workspace
+    (A, 16, -4),                 # too small
+    (A + 16, 1 << 30, -4),       # not 256-byte aligned
+])
+def test_backward_workspace_errors(ws_ptr, ws_bytes, code):
+    fa = _lib()
+    st = fa.fa_backward(A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 7 * A, 8 * A, 9 * A, 1, 2, 256, 64,
+                        0.125, 1, ws_ptr, ws_bytes, stream=0, check=False)
+    assert st == code
+
+
+def test_workspace_size_is_linear_in_n():
+    fa = _lib()
+    sizes = [fa.fa_backward_workspace_size(2, 4, n, 128) for n in (1024, 2048, 4096, 8192)]
+    diffs = [b - a for a, b in zip(sizes, sizes[1:])]
+    # doubling N doubles the increment: linear, not quadratic
+    assert diffs[1] == 2 * diffs[0] and diffs[2] == 2 * diffs[1]
+    # dQ accumulator + two padded row vectors, each rounded to 256 bytes
+    B, H, N, d = 2, 4, 1000, 80
+    np_ = 1024
+    up = lambda x: (x + 255) // 256 * 256
+    assert fa.fa_backward_workspace_size(B, H, N, d) == up(4 * B * H * N * d) + 2 * up(4 * B * H * np_)
+    assert fa.fa_backward_workspace_size(0, 1, 1, 64) == 0
+
+
+def test_flop_counter_matches_the_pages_worked_numbers():
+    # "FlashAttention-2" review, implementation-cost answer, (1) FLOPs:
+    # N = 1024, d = 64 -> forward 268,435,456, backward 671,088,640, total ~939e6.
+    assert perf.fwd_flops(1, 1, 1024, 64, False) == 268_435_456
+    assert perf.bwd_flops(1, 1, 1024, 64, False) == 671_088_640
+    total = perf.fwd_flops(1, 1, 1024, 64, False) + perf.bwd_flops(1, 1, 1024, 64, False)
+    assert int(total // 1e6) == 939  # 939.5e6, printed as "about 939 x 10^6"
+    assert perf.fwd_flops(1, 1, 1024, 64, True) == 268_435_456 / 2
+
+
+def test_workload_table():
+    w = workloads.WORKLOADS["causal_d128"]
+    assert (w.B, w.H, w.N, w.d, w.causal, w.backward) == (4, 16, 4096, 128, True, True)
+    assert abs(perf.fwd_flops(w.B, w.H, w.N, w.d, True) - 274.9e9) < 0.1e9
+    assert abs(perf.bwd_flops(w.B, w.H, w.N, w.d, True) - 687.2e9) < 0.1e9
+    w5 = workloads.WORKLOADS["gpt3_d80"]
+    assert w5.H * w5.d == w5.hidden == 2560
+
+
+def test_inputs_are_seeded_and_rounded():
+    w = workloads.WORKLOADS["fwd_d64"]
+    a = workloads.make_inputs(w, B=1, H=1, N=64)
+    b = workloads.make_inputs(w, B=1, H=1, N=64)
+    import torch
+    assert a["q"].dtype == torch.bfloat16
+    assert torch.equal(a["q"], b["q"]) and torch.equal(a["v"], b["v"])
+    p = workloads.make_inputs(workloads.WORKLOADS["gpt3_d80"], B=1, H=2, N=16)
+    assert p["q"].shape == (1, 2, 16, 80)
+    # projections of unit normals through N(0, 0.02^2) 2560-wide weights:
+    # entries have variance about 2560 * 0.02^2 = 1.02
+    big = workloads.make_inputs(workloads.WORKLOADS["gpt3_d80"], B=1, H=32, N=64)
+    var = big["k"].float().var().item()
+    assert 0.85 < var < 1.2
