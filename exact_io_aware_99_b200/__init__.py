@@ -6,18 +6,39 @@ used for device memory and streams.
 
 Low-level entry points (same names as the C ABI): ``fa_forward``,
 ``fa_forward_ex``, ``fa_backward``, ``fa_backward_ex``,
-``fa_backward_workspace_size``, ``fa_status_string``, ``fa_device_status``,
-``fa_set_wait_timeout_ns``, ``fa_selftest_wait_timeout``.
+``fa_backward_noalloc``, ``fa_backward_workspace_size``,
+``fa_status_string``, ``fa_device_status``, ``fa_set_wait_timeout_ns``,
+``fa_selftest_wait_timeout``.
 
 Convenience wrappers that allocate outputs with torch:
 ``attention_forward(q, k, v, scale=None, causal=False) -> (o, lse)`` and
 ``attention_backward(q, k, v, o, do, lse, scale=None, causal=False)
 -> (dq, dk, dv)``.
+
+The shared library is loaded on first use of any of these names (so the
+``build`` submodule can run before it exists); using them without the built
+library raises ImportError -- there is no fallback.
 """
-from ._native import (EXPORTS, FA_BF16, FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT,  # noqa: F401
-                      FA_ERR_INVALID_ARG, FA_ERR_MISALIGNED, FA_ERR_UNSUPPORTED,
-                      FA_ERR_WORKSPACE, FA_FP32, FA_OK, FaError, LIB_PATH,
-                      fa_backward, fa_backward_ex, fa_backward_workspace_size,
-                      fa_device_status, fa_forward, fa_forward_ex, fa_selftest_wait_timeout,
-                      fa_set_wait_timeout_ns, fa_status_string, library)
-from .api import attention_backward, attention_forward  # noqa: F401
+_NATIVE = {
+    "EXPORTS", "FA_BF16", "FA_FP32", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED",
+    "FA_ERR_MISALIGNED", "FA_ERR_WORKSPACE", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT",
+    "FA_NOALLOC_SCRATCH_BYTES", "FaError", "LIB_PATH", "library", "fa_forward",
+    "fa_forward_ex", "fa_backward", "fa_backward_ex", "fa_backward_noalloc",
+    "fa_backward_workspace_size", "fa_status_string", "fa_device_status",
+    "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout",
+}
+_API = {"attention_forward", "attention_backward"}
+
+
+def __getattr__(name):
+    if name in _NATIVE:
+        from . import _native
+        return getattr(_native, name)
+    if name in _API:
+        from . import api
+        return getattr(api, name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")
+
+
+def __dir__():
+    return sorted(set(globals()) | _NATIVE | _API)

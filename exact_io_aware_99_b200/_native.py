@@ -29,8 +29,11 @@ FA_FP32 = 1
 EXPORTS = (
     "fa_forward", "fa_forward_ex", "fa_backward_workspace_size", "fa_backward",
     "fa_backward_ex", "fa_status_string", "fa_last_cuda_error", "fa_device_status",
-    "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout",
+    "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_backward_noalloc",
 )
+
+# Size of the library's built-in scratch array used by fa_backward_noalloc.
+FA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class FaError(RuntimeError):
@@ -68,6 +71,8 @@ def _load() -> ctypes.CDLL:
     lib.fa_set_wait_timeout_ns.restype = None
     lib.fa_selftest_wait_timeout.argtypes = [P]
     lib.fa_selftest_wait_timeout.restype = I
+    lib.fa_backward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P]
+    lib.fa_backward_noalloc.restype = I
     return lib
 
 
@@ -156,3 +161,14 @@ def fa_set_wait_timeout_ns(ns: int) -> None:
 def fa_selftest_wait_timeout(stream=None, check=True) -> int:
     st = _lib.fa_selftest_wait_timeout(_stream(stream))
     return _check(st, "fa_selftest_wait_timeout", check)
+
+
+def fa_backward_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal,
+                        stream=None, check=True) -> int:
+    """fa_backward without a workspace argument: the scratch is the
+    library's built-in device array (FA_NOALLOC_SCRATCH_BYTES); nothing is
+    allocated.  For callers that cannot allocate device memory."""
+    st = _lib.fa_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                  int(bool(causal)), _stream(stream))
+    return _check(st, "fa_backward_noalloc", check)

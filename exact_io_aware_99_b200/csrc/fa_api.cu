@@ -289,3 +289,64 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free backward.
+//
+// The ordinary backward needs a caller-provided workspace.  Some callers have
+// no way to provide one: code running where every byte of device memory is
+// owned by some other allocator it cannot reach, plugins and callbacks that
+// are handed tensors but no means to reserve device memory, and
+// latency-bound loops that must never call cudaMalloc (it can synchronise the
+// whole device and take unbounded time).  fa_backward_noalloc serves them by
+// taking its scratch from a fixed array built into this library.
+//
+// The array lives in device memory of every GPU that loads the library, for
+// the life of the process.  All calls on a GPU share it and it keeps the
+// previous call's contents; the backward's preprocess kernel clears the dQ
+// accumulator and rewrites the row vectors on every call, so nothing carries
+// over between calls, but two calls whose kernels overlap on the GPU (for
+// example on two streams) race on the array.
+namespace {
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+fa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  if (g_noalloc_ptr[dev] == nullptr) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e);
+      g_noalloc_ptr[dev] = p;
+    }
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_backward_noalloc(const void* q, const void* k, const void* v,
+                                         const void* o, const void* dO, const float* lse,
+                                         void* dq, void* dk, void* dv, int B, int H, int N,
+                                         int d, float scale, int causal, void* stream) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || d > 128) return FA_ERR_INVALID_ARG;
+  if (ws_layout(B, H, N, d).total > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES))
+    return FA_ERR_WORKSPACE;  // the problem needs more scratch than the array holds
+  void* scratch = nullptr;
+  fa_status st = noalloc_scratch(&scratch);
+  if (st != FA_OK) return st;
+  return fa_backward_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, scratch,
+                        static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES), FA_BF16, stream);
+}

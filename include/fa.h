@@ -142,6 +142,33 @@ FA_API fa_status fa_backward_ex(const void* q, const void* k, const void* v,
                          void* workspace, size_t workspace_bytes,
                          fa_dtype dtype, void* stream);
 
+/*
+ * fa_backward_noalloc -- the bf16 backward of fa_backward, for callers that
+ * cannot allocate device memory or hand over a workspace: code whose device
+ * memory is entirely owned by another allocator, plugins and callbacks that
+ * receive tensors but cannot reserve scratch, and latency-bound loops that
+ * must not call cudaMalloc (it can synchronise the device).  The FlashAttention
+ * pages have no counterpart to this entry point; it is a convenience of this
+ * library.
+ *
+ * The scratch comes from a fixed device array of FA_NOALLOC_SCRATCH_BYTES
+ * built into the library (held on every GPU that loads it, until the process
+ * exits).  Problems whose workspace, fa_backward_workspace_size(B, H, N, d),
+ * exceeds that size are rejected with FA_ERR_WORKSPACE before anything runs.
+ * All calls on a GPU share the array: each call re-initialises what it needs,
+ * but calls whose kernels overlap on the GPU (e.g. on two streams) race.  The
+ * first call on each device looks up the array's device address (once, with
+ * that device current); make that first call before any stream capture.
+ * No device memory is allocated.  Arguments and results are those of
+ * fa_backward (bf16, d in {64, 80, 128}).
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (64u << 20)
+FA_API fa_status fa_backward_noalloc(const void* q, const void* k, const void* v,
+                              const void* o, const void* dO, const float* lse,
+                              void* dq, void* dk, void* dv,
+                              int B, int H, int N, int d, float scale, int causal,
+                              void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_API const char* fa_status_string(fa_status s);
 
