@@ -21,15 +21,19 @@
 //                 dP^T = V_j dO_i^T  -> TMEM cols [128,256)  (SS)
 //                 dV  += P^T dO_i    -> TMEM cols [256,256+d) (TS: P^T from TMEM)
 //                 dK  += dS^T Q_i    -> TMEM cols [384,384+d) (SS, dS^T from smem)
-//                 dQ_i = dS K_j      -> TMEM cols [0,d)      (SS, dS read MN-major)
+//                 dQ_i = dS K_j      -> TMEM cols [128,128+d) (SS, dS read MN-major)
 //   warps 0-3   one thread per key row: P^T = 2^(S^T c - LSE2) written back to
 //               TMEM as bf16 over S^T; dS^T = P^T o (dP^T - D) written to
 //               shared memory in the 128-byte-swizzled layout the MMAs read.
-//   warps 4-7   one thread per query row: read dQ_i from TMEM, scale, and add
-//               it to the fp32 dQ accumulator with 16-byte vector atomics;
-//               then the dK epilogue (warps 0-3 do dV).
-// TMEM holds 512 columns, so dQ_i reuses the S^T columns: S^T_{i+1} waits
-// until dQ_i has been read out.
+//   warps 4-7   one thread per query row: read dQ_i from TMEM, scale, stage
+//               it (fp32, 128-byte swizzled) in the dS buffer once the dK/dQ
+//               MMAs are done with it, and add it to the fp32 dQ accumulator
+//               with TMA tensor reductions (whole 128-byte lines); then the dK
+//               epilogue (warps 0-3 do dV).
+// TMEM holds 512 columns, so dQ_i reuses the dP^T columns: S^T_{i+1} is
+// issued right behind dQ_i and overlaps the dQ readout; dP^T_{i+1} waits for
+// the readout.  CTAs run group-major (a few heads at a time, so their K, V,
+// Q, dO and dQ accumulator stay in L2), longest-first inside a group.
 #include <cuda_bf16.h>
 
 #include "fa_internal.h"
@@ -57,6 +61,8 @@ struct Cfg {
   static constexpr int DS_BYTES = 2 * BLK;        // 128 keys x 128 queries bf16
   static constexpr int BAR_OFF = DS_OFF + DS_BYTES;
   static constexpr int NBAR = 16;
+  static constexpr int NSUB = (D + 31) / 32;      // 32-column fp32 dQ sub-tiles
+  static_assert(DS_BYTES >= 4 * 2 * 4096, "dQ staging: 4 warps x 2 sub-tiles of 32x32 fp32");
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
   static constexpr int KSTEPS = D / 16;
@@ -95,9 +101,10 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const float* __restrict__ dvec, const float* __restrict__ lse2,
-               float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
-               __nv_bfloat16* __restrict__ dv, int N, float scale, float scale_log2, WaitCtl ctl) {
+               const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ dvec,
+               const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dk,
+               __nv_bfloat16* __restrict__ dv, int N, int BH, int group, float scale,
+               float scale_log2, WaitCtl ctl) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -113,17 +120,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* dp_full = bars + 8;
   uint64_t* p_full = bars + 9;
   uint64_t* ds_full = bars + 10;
-  uint64_t* dq_full = bars + 11;   // also "dS buffer free"
-  uint64_t* dq_empty = bars + 12;
-  uint64_t* kv_done = bars + 13;
+  uint64_t* dq_full = bars + 11;
+  uint64_t* dq_empty = bars + 12;  // dQ read out of TMEM (dP^T columns free)
+  uint64_t* ds_free = bars + 13;   // dQ staging done with the dS buffer
+  uint64_t* kv_done = bars + 14;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int bh = blockIdx.x;
-  const int j = blockIdx.y;  // key tile; j = 0 has the most work when causal
   const int n_q = (N + kBN - 1) / kBN;
+  // Group-major order: `group` heads at a time, and inside a group key tile
+  // j ascending (j = 0 has the most work when causal), head fastest.
+  int bh, j;
+  {
+    const int per_group = group * n_q;
+    const int g = static_cast<int>(blockIdx.x) / per_group;
+    const int r = static_cast<int>(blockIdx.x) - g * per_group;
+    const int gh = min(group, BH - g * group);
+    j = r / gh;
+    bh = g * group + (r - j * gh);
+  }
   const int Np = n_q * kBN;
   const int i_start = CAUSAL ? j : 0;
   const int n_iter = n_q - i_start;
@@ -141,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(ds_full, kBM);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, kBN);
+    mbar_init(ds_free, 4);
     mbar_init(kv_done, 1);
     *abort = 0;
     fence_barrier_init();
@@ -205,15 +223,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t k_addr = sbase + C::K_OFF;
       const uint32_t v_addr = sbase + C::V_OFF;
       const uint32_t ds_addr = sbase + C::DS_OFF;
-      bool ok = mbar_wait(kv_full, 0, abort, ctl, kSiteBwdMma);
-      for (int it = 0; ok && it < n_iter; ++it) {
+      auto issue_s = [&](int it) -> bool {  // S^T = K_j Q_i^T -> cols [0,128)
         const int st = it & 1;
-        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1;
-        const uint32_t q_addr = sbase + C::Q_OFF + st * C::TILE;
-        const uint32_t do_addr = sbase + C::DO_OFF + st * C::TILE;
-        if (!mbar_wait(q_full + st, ph, abort, ctl, kSiteBwdMma)) break;
-        if (it > 0 && !mbar_wait(dq_empty, (it - 1) & 1, abort, ctl, kSiteBwdMma)) break;
+        if (!mbar_wait(q_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
+          return false;
         tc_fence_after();
+        const uint32_t q_addr = sbase + C::Q_OFF + st * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
@@ -221,7 +236,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                  sdesc_sw128(q_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full);
+        return true;
+      };
+      bool ok = mbar_wait(kv_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0);
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1;
+        const uint32_t q_addr = sbase + C::Q_OFF + st * C::TILE;
+        const uint32_t do_addr = sbase + C::DO_OFF + st * C::TILE;
+        // dP^T = V_j dO_i^T -> cols [128,256), once dQ_{i-1} has been read out.
         if (!mbar_wait(do_full + st, ph, abort, ctl, kSiteBwdMma)) break;
+        if (it > 0 && !mbar_wait(dq_empty, (it - 1) & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
@@ -230,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  sdesc_sw128(do_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
         }
         mma_commit(dp_full);
+        // dV += P^T dO_i, P^T read from TMEM.
         if (!mbar_wait(p_full, it & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
 #pragma unroll
@@ -237,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + kColDV, tmem + kColS + kk * 8,
                  sdesc_sw128(do_addr + kk * 2048, C::BLK, 1024), kIdescAcc,
                  (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q_i and dQ_i = dS K_j (into the dP^T columns).
         if (!mbar_wait(ds_full, it & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
 #pragma unroll
@@ -248,10 +275,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_ss(tmem + kColS, sdesc_sw128(ds_addr + kk * 2048, C::BLK, 1024),
+          mma_ss(tmem + kColDP, sdesc_sw128(ds_addr + kk * 2048, C::BLK, 1024),
                  sdesc_sw128(k_addr + kk * 2048, C::BLK, 1024), kIdescDq, kk > 0 ? 1u : 0u);
         mma_commit(dq_full);
         mma_commit(qdo_empty + st);
+        // S^T of the next query tile overlaps the dQ readout.
+        if (it + 1 < n_iter) ok = issue_s(it + 1);
       }
       mma_commit(kv_done);
     }
@@ -303,8 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(p_full);
 
-      // dS^T needs the dS buffer back from iteration it-1 and dP^T of this one.
-      if (it > 0 && !wait_all(dq_full, (it - 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
+      // dS^T needs the dS buffer back (dK/dQ MMAs and the dQ staging of
+      // iteration it-1 are done with it) and dP^T of this iteration.
+      if (it > 0 && !wait_all(ds_free, (it - 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
         ok = false;
         break;
       }
@@ -360,34 +390,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // --------------------------------------------- dQ readout (warps 4..7)
+    const int wq = warp - 4;           // TMEM lane quarter: query rows 32*wq..
     const int qr = threadIdx.x - 128;  // query row == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    // Per-warp staging: two 32 x 32 fp32 sub-tiles (4 KB each, 128-byte
+    // swizzled) inside the dS buffer.
+    uint8_t* stage = smem + C::DS_OFF + wq * 8192;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
-      const int q_idx = (i_start + it) * kBN + qr;
+      const int q0 = (i_start + it) * kBN;
       if (!wait_all(dq_full, it & 1, abort, ctl, kSiteBwdDq)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float4* dst = reinterpret_cast<float4*>(dq_acc + (static_cast<size_t>(bh) * N + q_idx) * D);
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t v16[16];
-        tmem_ld16(lane_base + kColS + c * 16, v16);
-        tmem_wait_ld();
-        if (q_idx < N) {
+      for (int pass = 0; pass < (C::NSUB + 1) / 2; ++pass) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            atomicAdd(dst + c * 4 + e, make_float4(__uint_as_float(v16[4 * e]) * scale,
-                                                   __uint_as_float(v16[4 * e + 1]) * scale,
-                                                   __uint_as_float(v16[4 * e + 2]) * scale,
-                                                   __uint_as_float(v16[4 * e + 3]) * scale));
+        for (int sl = 0; sl < 2; ++sl) {
+          const int sub = 2 * pass + sl;
+          if (sub < C::NSUB) {
+            uint32_t v[32];
+            tmem_ld32(lane_base + kColDP + sub * 32, v);
+            tmem_wait_ld();
+            uint8_t* rowp = stage + sl * 4096 + lane * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float4 f = make_float4(__uint_as_float(v[4 * c]) * scale,
+                                           __uint_as_float(v[4 * c + 1]) * scale,
+                                           __uint_as_float(v[4 * c + 2]) * scale,
+                                           __uint_as_float(v[4 * c + 3]) * scale);
+              *reinterpret_cast<float4*>(rowp + ((c ^ (lane & 7)) * 16)) = f;
+            }
+          }
         }
+        if (2 * pass + 2 >= C::NSUB) {
+          // Last TMEM read of dQ_i: release the dP^T columns.
+          tc_fence_before();
+          mbar_arrive(dq_empty);
+        }
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          const int y = q0 + wq * 32;
+          if (y < N) {
+#pragma unroll
+            for (int sl = 0; sl < 2; ++sl)
+              if (2 * pass + sl < C::NSUB)
+                tma_reduce_add_3d(&tm_dq, stage + sl * 4096, (2 * pass + sl) * 32, y, bh);
+          }
+          bulk_commit();
+          bulk_wait_read_all();
+        }
+        __syncwarp();
       }
-      tc_fence_before();
-      mbar_arrive(dq_empty);
+      if (lane == 0) mbar_arrive(ds_free);
+      (void)qr;
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
     // dK epilogue
     if (ok && wait_all(kv_done, 0, abort, ctl, kSiteBwdEpilogue)) {
       tc_fence_after();
@@ -421,8 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool CAUSAL>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const CUtensorMap& tdo, const float* dvec, const float* lse2, float* dq_acc,
-                   void* dk, void* dv, int BH, int N, float scale, const Launch& L) {
+                   const CUtensorMap& tdo, const CUtensorMap& tdq, const float* dvec,
+                   const float* lse2, void* dk, void* dv, int BH, int N, float scale,
+                   const Launch& L) {
   using C = Cfg<D>;
   static bool configured = false;
   if (!configured) {
@@ -431,39 +493,41 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  dim3 grid(BH, (N + kBM - 1) / kBM);
+  const int n_kv = (N + kBM - 1) / kBM;
+  // Heads per group: keep a group's K, V, Q, dO (bf16) and dQ accumulator
+  // (fp32), 12 N d bytes per head, within ~48 MB of the 126 MB L2.
+  const long long per_head = 12LL * N * D;
+  int group = static_cast<int>((48LL << 20) / (per_head > 0 ? per_head : 1));
+  group = group < 1 ? 1 : (group > BH ? BH : group);
+  const long long blocks = static_cast<long long>(BH) * n_kv;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   WaitCtl ctl{L.status, L.limit_ns};
-  bwd_kernel<D, CAUSAL><<<grid, kThreads, C::SMEM, L.stream>>>(
-      tq, tk, tv, tdo, dvec, lse2, dq_acc, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), N, scale, scale * 1.4426950408889634f, ctl);
+  bwd_kernel<D, CAUSAL><<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
+      tq, tk, tv, tdo, tdq, dvec, lse2, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv), N, BH, group, scale, scale * 1.4426950408889634f, ctl);
   return cudaGetLastError();
 }
 
 }  // namespace bwd
 
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tdo, const float* dvec, const float* lse2,
-                             float* dq_acc, void* dk, void* dv, int BH, int N, int d, float scale,
-                             int causal, const Launch& L) {
+                             const CUtensorMap& tdo, const CUtensorMap& tdq, const float* dvec,
+                             const float* lse2, void* dk, void* dv, int BH, int N, int d,
+                             float scale, int causal, const Launch& L) {
+#define FA_BWD_CASE(DD)                                                                     \
+  case DD:                                                                                  \
+    return causal ? bwd::launch<DD, true>(tq, tk, tv, tdo, tdq, dvec, lse2, dk, dv, BH, N,  \
+                                          scale, L)                                         \
+                  : bwd::launch<DD, false>(tq, tk, tv, tdo, tdq, dvec, lse2, dk, dv, BH, N, \
+                                           scale, L);
   switch (d) {
-    case 64:
-      return causal ? bwd::launch<64, true>(tq, tk, tv, tdo, dvec, lse2, dq_acc, dk, dv, BH, N,
-                                            scale, L)
-                    : bwd::launch<64, false>(tq, tk, tv, tdo, dvec, lse2, dq_acc, dk, dv, BH, N,
-                                             scale, L);
-    case 80:
-      return causal ? bwd::launch<80, true>(tq, tk, tv, tdo, dvec, lse2, dq_acc, dk, dv, BH, N,
-                                            scale, L)
-                    : bwd::launch<80, false>(tq, tk, tv, tdo, dvec, lse2, dq_acc, dk, dv, BH, N,
-                                             scale, L);
-    case 128:
-      return causal ? bwd::launch<128, true>(tq, tk, tv, tdo, dvec, lse2, dq_acc, dk, dv, BH, N,
-                                             scale, L)
-                    : bwd::launch<128, false>(tq, tk, tv, tdo, dvec, lse2, dq_acc, dk, dv, BH, N,
-                                              scale, L);
+    FA_BWD_CASE(64)
+    FA_BWD_CASE(80)
+    FA_BWD_CASE(128)
     default:
       return cudaErrorInvalidValue;
   }
+#undef FA_BWD_CASE
 }
 
 }  // namespace fa

@@ -25,7 +25,8 @@
 //               corrections rare after the first tiles.  They also run the
 //               epilogue (O / l -> bf16, LSE).
 // Causal: tiles above the diagonal are never loaded; only the diagonal tile
-// and a ragged last tile are masked.  CTAs are launched longest-first.
+// and a ragged last tile are masked.  CTAs run group-major (a few heads at a
+// time, so their K and V stay in L2), longest-first inside a group.
 #include <cuda_bf16.h>
 
 #include "fa_internal.h"
@@ -75,7 +76,8 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-               float* __restrict__ lse, int N, float scale_log2, WaitCtl ctl) {
+               float* __restrict__ lse, int N, int BH, int group, float scale_log2,
+               WaitCtl ctl) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -96,9 +98,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int bh = blockIdx.x;
-  const int qt = static_cast<int>(gridDim.y) - 1 - static_cast<int>(blockIdx.y);
   const int n_kv_all = (N + kBN - 1) / kBN;
+  // Group-major order: `group` heads at a time (their K and V stay in L2),
+  // and inside a group the longest query tiles first, head fastest.
+  int bh, qt;
+  {
+    const int per_group = group * n_kv_all;
+    const int g = static_cast<int>(blockIdx.x) / per_group;
+    const int r = static_cast<int>(blockIdx.x) - g * per_group;
+    const int gh = min(group, BH - g * group);
+    const int t = r / gh;
+    qt = n_kv_all - 1 - t;
+    bh = g * group + (r - t * gh);
+  }
   const int n_kv = CAUSAL ? min(qt + 1, n_kv_all) : n_kv_all;
 
   if (threadIdx.x == 0) {
@@ -363,11 +375,17 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     configured = true;
   }
   const int n_qt = (N + kBM - 1) / kBM;
-  dim3 grid(BH, n_qt);
+  // Heads per group: keep a group's Q, K, V and O (8 N d bytes per head)
+  // within ~48 MB of the 126 MB L2.
+  const long long per_head = 8LL * N * D;
+  int group = static_cast<int>((48LL << 20) / (per_head > 0 ? per_head : 1));
+  group = group < 1 ? 1 : (group > BH ? BH : group);
+  const long long blocks = static_cast<long long>(BH) * n_qt;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};
-  fwd_kernel<D, CAUSAL><<<grid, kThreads, C::SMEM, L.stream>>>(
-      tq, tk, tv, static_cast<__nv_bfloat16*>(o), lse, N, scale_log2, ctl);
+  fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
+      tq, tk, tv, static_cast<__nv_bfloat16*>(o), lse, N, BH, group, scale_log2, ctl);
   return cudaGetLastError();
 }
 

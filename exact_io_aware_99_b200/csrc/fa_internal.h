@@ -43,10 +43,12 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
                              void* o, float* lse, int BH, int N, int d, float scale, int causal,
                              const Launch& L);
 
+// tdq: the fp32 dQ accumulator [BH, N, d] as 3-D {d, N, BH}, box {32, 32, 1},
+// 128-byte swizzle (target of the TMA reductions).
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tdo, const float* dvec, const float* lse2,
-                             float* dq_acc, void* dk, void* dv, int BH, int N, int d, float scale,
-                             int causal, const Launch& L);
+                             const CUtensorMap& tdo, const CUtensorMap& tdq, const float* dvec,
+                             const float* lse2, void* dk, void* dv, int BH, int N, int d,
+                             float scale, int causal, const Launch& L);
 
 // --- helpers shared by both dtypes (fa_simt.cu) ---------------------------
 // D = rowsum(dO o O) (fp32, padded rows = 0), lse2 = LSE * log2(e) (padded
