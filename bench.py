@@ -313,7 +313,7 @@ def run_ours(args, peaks, peak_kind):
         "frac_of_sustained_peak": round(value / ws / peak_s, 4),
         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json bf16_tflops burst {peak}, "
                        f"sustained {peak_s})",
-        "roofline": {"kernel": "fa_backward (preprocess + dK/dV/dQ kernel + dQ convert)",
+        "roofline": {"kernel": "fa_backward (preprocess + dK/dV kernel + dQ kernel)",
                      "bound": "tensor", "achieved": round(bwd_tf, 3), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(bwd_tf / peak, 4),
                      "traffic": traffic,

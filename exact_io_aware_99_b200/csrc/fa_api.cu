@@ -106,26 +106,6 @@ fa_status make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
   return FA_OK;
 }
 
-// fp32 [BH, N, d] as 3-D {d, N, BH}; box {32, 32, 1}; 128-byte swizzle
-// (the backward's dQ accumulator, written with TMA reductions).
-fa_status make_map_f32_acc(CUtensorMap* m, const void* base, int BH, int N, int d) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
-                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 4};
-  cuuint32_t box[3] = {32, 32, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    g_last_cuda_error = static_cast<int>(r);
-    return FA_ERR_CUDA;
-  }
-  return FA_OK;
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 fa_status check_common(int B, int H, int N, int d, float scale, fa_dtype dtype) {
@@ -147,7 +127,7 @@ fa_status check_common(int B, int H, int N, int d, float scale, fa_dtype dtype) 
 }
 
 struct WsLayout {
-  size_t dq_off, dvec_off, lse2_off, total;
+  size_t dvec_off, lse2_off, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -155,10 +135,11 @@ size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 WsLayout ws_layout(int B, int H, int N, int d) {
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t np = static_cast<size_t>(fa::round_up(N, fa::kTileRows));
+  (void)N;
+  (void)d;
   WsLayout w;
-  w.dq_off = 0;
-  w.dvec_off = up256(bh * N * d * sizeof(float));
-  w.lse2_off = w.dvec_off + up256(bh * np * sizeof(float));
+  w.dvec_off = 0;
+  w.lse2_off = up256(bh * np * sizeof(float));
   w.total = w.lse2_off + up256(bh * np * sizeof(float));
   return w;
 }
@@ -272,12 +253,11 @@ fa_status fa_backward_ex(const void* q, const void* k, const void* v, const void
   const int BH = B * H;
   const int cz = causal ? 1 : 0;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* dq_acc = reinterpret_cast<float*>(ws + w.dq_off);
   float* dvec = reinterpret_cast<float*>(ws + w.dvec_off);
   float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
   cudaError_t e;
   if (dtype == FA_FP32) {
-    e = fa::launch_bwd_preprocess(o, dO, lse, dvec, nullptr, nullptr, BH, N, d, 0, L);
+    e = fa::launch_bwd_preprocess(o, dO, lse, dvec, nullptr, BH, N, d, 0, L);
     if (e != cudaSuccess) return cuda_fail(e);
     e = fa::launch_bwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                            static_cast<const float*>(v), static_cast<const float*>(dO), lse, dvec,
@@ -287,17 +267,14 @@ fa_status fa_backward_ex(const void* q, const void* k, const void* v, const void
   }
   st = get_encoder();
   if (st != FA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo;
   if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tdo, dO, BH, N, d)) != FA_OK) return st;
-  if ((st = make_map_f32_acc(&tdq, dq_acc, BH, N, d)) != FA_OK) return st;
-  e = fa::launch_bwd_preprocess(o, dO, lse, dvec, lse2, dq_acc, BH, N, d, 1, L);
+  e = fa::launch_bwd_preprocess(o, dO, lse, dvec, lse2, BH, N, d, 1, L);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, tdq, dvec, lse2, dk, dv, BH, N, d, scale, cz, L);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = fa::launch_dq_convert_bf16(dq_acc, dq, static_cast<size_t>(BH) * N * d, L);
+  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, d, scale, cz, L);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 

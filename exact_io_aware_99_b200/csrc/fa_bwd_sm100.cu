@@ -10,30 +10,35 @@
 // (The page prints dS as "dP.P - P.(dP.P^T)" and drops the scale; the
 // row-wise softmax Jacobian and the chain-rule scale are the reading used.)
 //
-// B200 design: one CTA per (head, 128-key tile K_j/V_j), looping over the
-// query tiles Q_i that see it (all of them, or i >= j when causal), so the
-// work is parallel over batch, head and sequence as FA2 prescribes
-// ("FlashAttention-2" review, results answer, parallelism over sequence
-// length).  10 warps:
-//   warp 8      TMA producer: K_j, V_j once; Q_i and dO_i into a 2-stage ring.
-//   warp 9      TMEM allocator and single-thread MMA issuer, per Q tile:
-//                 S^T  = K_j Q_i^T   -> TMEM cols [0,128)    (SS)
-//                 dP^T = V_j dO_i^T  -> TMEM cols [128,256)  (SS)
-//                 dV  += P^T dO_i    -> TMEM cols [256,256+d) (TS: P^T from TMEM)
-//                 dK  += dS^T Q_i    -> TMEM cols [384,384+d) (SS, dS^T from smem)
-//                 dQ_i = dS K_j      -> TMEM cols [128,128+d) (SS, dS read MN-major)
-//   warps 0-3   one thread per key row: P^T = 2^(S^T c - LSE2) written back to
-//               TMEM as bf16 over S^T; dS^T = P^T o (dP^T - D) written to
-//               shared memory in the 128-byte-swizzled layout the MMAs read.
-//   warps 4-7   one thread per query row: read dQ_i from TMEM, scale, stage
-//               it (fp32, 128-byte swizzled) in the dS buffer once the dK/dQ
-//               MMAs are done with it, and add it to the fp32 dQ accumulator
-//               with TMA tensor reductions (whole 128-byte lines); then the dK
-//               epilogue (warps 0-3 do dV).
-// TMEM holds 512 columns, so dQ_i reuses the dP^T columns: S^T_{i+1} is
-// issued right behind dQ_i and overlaps the dQ readout; dP^T_{i+1} waits for
-// the readout.  CTAs run group-major (a few heads at a time, so their K, V,
-// Q, dO and dQ accumulator stay in L2), longest-first inside a group.
+// B200 design: two kernels, each parallel over batch, head and sequence (the
+// FA2 review's results answer: parallelism over the sequence length), and
+// each keeping every MMA operand it can in tensor memory (TMEM), because the
+// shared-memory port (128 B/clk/SM) is what limits a 128 x 128 tile pair:
+//
+//  dK/dV kernel -- one CTA per (head, 128-key tile K_j, V_j), looping over the
+//  query tiles Q_i that see it.  Per Q tile:
+//      S^T  = K_j Q_i^T   (SS)  -> TMEM A = cols [0,128)
+//      dP^T = V_j dO_i^T  (SS)  -> TMEM B = cols [128,256)
+//      softmax warps: P^T = 2^(S^T c - LSE2) into already-read columns of A,
+//        dS^T = P^T o (dP^T - D) into already-read columns of B (bf16)
+//      dV += P^T dO_i     (TS, P^T from TMEM)  -> cols [256,256+d)
+//      dK += dS^T Q_i     (TS, dS^T from TMEM) -> cols [384,384+d)
+//    issued as S_0, dP_0, dV_0, S_1, dK_0, dP_1, dV_1, S_2, dK_1, ... so the
+//    softmax forms P_{i+1} while the tensor core runs dK_i and dP_{i+1}.
+//  dQ kernel -- one CTA per (head, 128-query tile Q_i), looping over the key
+//  tiles K_j it sees.  Per key tile:
+//      S  = Q_i K_j^T     (SS)  -> TMEM S buffer j%2 (double-buffered)
+//      dP = dO_i V_j^T    (SS)  -> cols [256,384)
+//      softmax warps: dS = P o (dP - D), bf16, into read columns of S
+//      dQ += dS K_j       (TS, dS from TMEM) -> cols [384,384+d)
+//  and dQ is written once, in bf16, at the end: no atomics and no fp32 dQ
+//  buffer, at the price of recomputing S and dP (7 tile MMAs per tile pair
+//  instead of 5).
+// Warp roles (both kernels, 10 warps): warps 0-3 and 4-7 are two softmax
+// warpgroups splitting the 128 columns of every tile in halves (one thread
+// per TMEM lane), warp 8 is the TMA producer, warp 9 the TMEM allocator and
+// single-thread MMA issuer.  CTAs run group-major (a few heads at a time, so
+// their operands stay in L2), longest-first inside a group.
 #include <cuda_bf16.h>
 
 #include "fa_internal.h"
@@ -42,32 +47,17 @@
 namespace fa {
 namespace bwd {
 
-constexpr int kBM = 128;  // keys per CTA (TMEM lanes of S^T, dP^T, dK, dV)
-constexpr int kBN = 128;  // queries per inner tile
+constexpr int kT = 128;  // rows of every tile (keys or queries)
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 
 template <int D>
-struct Cfg {
+struct Shape {
   static constexpr int NB = (D + 63) / 64;
-  static constexpr int BLK = 64 * 128 * 2;  // one 128-row x 64-col bf16 swizzle block
+  static constexpr int BLK = 64 * kT * 2;  // one 128-row x 64-col bf16 swizzle block
   static constexpr int TILE = NB * BLK;
-  static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = K_OFF + TILE;
-  static constexpr int Q_OFF = V_OFF + TILE;      // [2] stages
-  static constexpr int DO_OFF = Q_OFF + 2 * TILE; // [2] stages
-  static constexpr int DS_OFF = DO_OFF + 2 * TILE;
-  static constexpr int DS_BYTES = 2 * BLK;        // 128 keys x 128 queries bf16
-  static constexpr int BAR_OFF = DS_OFF + DS_BYTES;
-  static constexpr int NBAR = 16;
-  static constexpr int NSUB = (D + 31) / 32;      // 32-column fp32 dQ sub-tiles
-  static_assert(DS_BYTES >= 4 * 2 * 4096, "dQ staging: 4 warps x 2 sub-tiles of 32x32 fp32");
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int SMEM = MISC_OFF + 16 + 1024;
   static constexpr int KSTEPS = D / 16;
   static_assert(D % 16 == 0 && D <= 128, "head dim must be a multiple of 16, <= 128");
-  static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
@@ -88,24 +78,77 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, w);
 }
 
-// Store 8 consecutive bf16 (one 16-byte chunk) of row `row`, chunk `chunk`
-// (0..15 over 128 columns) of a 128-row tile in the 128-byte-swizzled layout:
-// 64-column blocks of 128 x 128 B, chunk index XOR (row mod 8).
-__device__ __forceinline__ void st_sw128(uint8_t* tile, int row, int chunk, uint4 val) {
-  const int blk = chunk >> 3;
-  const int c = (chunk & 7) ^ (row & 7);
-  *reinterpret_cast<uint4*>(tile + blk * (64 * 128 * 2) + row * 128 + c * 16) = val;
+// (head, tile) of this CTA in group-major order: `group` heads at a time;
+// inside a group tile index t ascending, head fastest.
+__device__ __forceinline__ void group_major(int n_tiles, int BH, int group, int& bh, int& t) {
+  const int per_group = group * n_tiles;
+  const int g = static_cast<int>(blockIdx.x) / per_group;
+  const int r = static_cast<int>(blockIdx.x) - g * per_group;
+  const int gh = min(group, BH - g * group);
+  t = r / gh;
+  bh = g * group + (r - t * gh);
 }
+
+// Store one row of a tile from TMEM columns [taddr, taddr + D) (fp32, times
+// `mul`) to global memory as bf16, 16 columns per step; the steps alternate
+// between the two softmax warpgroups (h = 0, 1).
+template <int D>
+__device__ __forceinline__ void store_row_bf16(uint32_t taddr, float mul, __nv_bfloat16* row,
+                                               bool valid, int h) {
+#pragma unroll
+  for (int c = 0; c < D / 16; ++c) {
+    if ((c & 1) != h) continue;
+    uint32_t v16[16];
+    tmem_ld16(taddr + c * 16, v16);
+    tmem_wait_ld();
+    uint32_t pk[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      pk[e] = pack_bf16(__uint_as_float(v16[2 * e]) * mul, __uint_as_float(v16[2 * e + 1]) * mul);
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(row + c * 16);
+      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+  }
+}
+
+// =========================================================================
+// dK / dV
+// =========================================================================
+
+template <int D>
+struct KvCfg : Shape<D> {
+  using S = Shape<D>;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + S::TILE;
+  static constexpr int Q_OFF = V_OFF + S::TILE;       // [2] stages
+  static constexpr int DO_OFF = Q_OFF + 2 * S::TILE;  // [2] stages
+  // [2] stages of the query tile's LSE2 (512 B) then D (512 B)
+  static constexpr int VEC_OFF = DO_OFF + 2 * S::TILE;
+  static constexpr int BAR_OFF = VEC_OFF + 2 * 1024;
+  static constexpr int NBAR = 16;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// TMEM columns of the dK/dV kernel.  Region A holds S^T, region B dP^T;
+// softmax warpgroup h reads S^T columns [64h, 64h+64) and writes its P^T
+// (bf16 pairs) into [64h, 64h+32), then reads dP^T columns [128+64h, +64)
+// and writes its dS^T into [128+64h, 128+64h+32).
+constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvColDV = 256, kKvColDK = 384;
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ dvec,
-               const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dk,
-               __nv_bfloat16* __restrict__ dv, int N, int BH, int group, float scale,
-               float scale_log2, WaitCtl ctl) {
-  using C = Cfg<D>;
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ dvec,
+                    const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dk,
+                    __nv_bfloat16* __restrict__ dv, int N, int BH, int group, float scale,
+                    float scale_log2, WaitCtl ctl) {
+  using C = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -118,32 +161,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qdo_empty = bars + 5;  // [2]
   uint64_t* s_full = bars + 7;
   uint64_t* dp_full = bars + 8;
-  uint64_t* p_full = bars + 9;
-  uint64_t* ds_full = bars + 10;
-  uint64_t* dq_full = bars + 11;
-  uint64_t* dq_empty = bars + 12;  // dQ read out of TMEM (dP^T columns free)
-  uint64_t* ds_free = bars + 13;   // dQ staging done with the dS buffer
-  uint64_t* kv_done = bars + 14;
+  uint64_t* p_full = bars + 9;     // both softmax warpgroups wrote P^T
+  uint64_t* ds_full = bars + 10;   // both wrote dS^T (and are done with S^T, dP^T)
+  uint64_t* kv_done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int n_q = (N + kBN - 1) / kBN;
-  // Group-major order: `group` heads at a time, and inside a group key tile
-  // j ascending (j = 0 has the most work when causal), head fastest.
+  const int n_t = (N + kT - 1) / kT;
+  const int Np = n_t * kT;
   int bh, j;
-  {
-    const int per_group = group * n_q;
-    const int g = static_cast<int>(blockIdx.x) / per_group;
-    const int r = static_cast<int>(blockIdx.x) - g * per_group;
-    const int gh = min(group, BH - g * group);
-    j = r / gh;
-    bh = g * group + (r - j * gh);
-  }
-  const int Np = n_q * kBN;
+  group_major(n_t, BH, group, bh, j);  // j = 0 first: most query tiles when causal
   const int i_start = CAUSAL ? j : 0;
-  const int n_iter = n_q - i_start;
+  const int n_iter = n_t - i_start;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -154,11 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, kBM);
-    mbar_init(ds_full, kBM);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_empty, kBN);
-    mbar_init(ds_free, 4);
+    mbar_init(p_full, 2 * kT);
+    mbar_init(ds_full, 2 * kT);
     mbar_init(kv_done, 1);
     *abort = 0;
     fence_barrier_init();
@@ -183,20 +211,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
 #pragma unroll
       for (int b = 0; b < C::NB; ++b) {
-        tma_load_3d(&tm_k, kv_full, smem + C::K_OFF + b * C::BLK, b * 64, j * kBM, bh);
-        tma_load_3d(&tm_v, kv_full, smem + C::V_OFF + b * C::BLK, b * 64, j * kBM, bh);
+        tma_load_3d(&tm_k, kv_full, smem + C::K_OFF + b * C::BLK, b * 64, j * kT, bh);
+        tma_load_3d(&tm_v, kv_full, smem + C::V_OFF + b * C::BLK, b * 64, j * kT, bh);
       }
       for (int it = 0; it < n_iter; ++it) {
         const int st = it & 1;
         const uint32_t u = static_cast<uint32_t>(it >> 1);
         if (it >= 2 && !mbar_wait(qdo_empty + st, (u - 1) & 1, abort, ctl, kSiteBwdProducer))
           break;
-        const int y = (i_start + it) * kBN;
-        mbar_arrive_expect_tx(q_full + st, C::TILE);
+        const int y = (i_start + it) * kT;
+        mbar_arrive_expect_tx(q_full + st, C::TILE + 1024);
 #pragma unroll
         for (int b = 0; b < C::NB; ++b)
           tma_load_3d(&tm_q, q_full + st, smem + C::Q_OFF + st * C::TILE + b * C::BLK, b * 64, y,
                       bh);
+        const size_t vrow = static_cast<size_t>(bh) * Np + y;
+        bulk_load_1d(smem + C::VEC_OFF + st * 1024, lse2 + vrow, 512, q_full + st);
+        bulk_load_1d(smem + C::VEC_OFF + st * 1024 + 512, dvec + vrow, 512, q_full + st);
         mbar_arrive_expect_tx(do_full + st, C::TILE);
 #pragma unroll
         for (int b = 0; b < C::NB; ++b)
@@ -217,13 +248,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescSq = idesc_bf16(kBM, kBN, 0, 0);  // S^T, dP^T
-      constexpr uint32_t kIdescAcc = idesc_bf16(kBM, D, 0, 1);   // dV, dK (B MN-major)
-      constexpr uint32_t kIdescDq = idesc_bf16(kBN, D, 1, 1);    // dQ (A and B MN-major)
+      constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S^T, dP^T
+      constexpr uint32_t kIdescAcc = idesc_bf16(kT, D, 0, 1);  // dV, dK (B MN-major)
       const uint32_t k_addr = sbase + C::K_OFF;
       const uint32_t v_addr = sbase + C::V_OFF;
-      const uint32_t ds_addr = sbase + C::DS_OFF;
-      auto issue_s = [&](int it) -> bool {  // S^T = K_j Q_i^T -> cols [0,128)
+      auto issue_s = [&](int it) -> bool {  // S^T = K_j Q_i^T -> region A
         const int st = it & 1;
         if (!mbar_wait(q_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
           return false;
@@ -232,243 +261,164 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kColS, sdesc_sw128(k_addr + off, 16, 1024),
+          mma_ss(tmem + kKvColS, sdesc_sw128(k_addr + off, 16, 1024),
                  sdesc_sw128(q_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full);
         return true;
       };
-      bool ok = mbar_wait(kv_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0);
-      for (int it = 0; ok && it < n_iter; ++it) {
+      auto issue_dp = [&](int it) -> bool {  // dP^T = V_j dO_i^T -> region B
         const int st = it & 1;
-        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1;
-        const uint32_t q_addr = sbase + C::Q_OFF + st * C::TILE;
-        const uint32_t do_addr = sbase + C::DO_OFF + st * C::TILE;
-        // dP^T = V_j dO_i^T -> cols [128,256), once dQ_{i-1} has been read out.
-        if (!mbar_wait(do_full + st, ph, abort, ctl, kSiteBwdMma)) break;
-        if (it > 0 && !mbar_wait(dq_empty, (it - 1) & 1, abort, ctl, kSiteBwdMma)) break;
+        if (!mbar_wait(do_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
+          return false;
         tc_fence_after();
+        const uint32_t do_addr = sbase + C::DO_OFF + st * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kColDP, sdesc_sw128(v_addr + off, 16, 1024),
+          mma_ss(tmem + kKvColDP, sdesc_sw128(v_addr + off, 16, 1024),
                  sdesc_sw128(do_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
         }
         mma_commit(dp_full);
-        // dV += P^T dO_i, P^T read from TMEM.
+        return true;
+      };
+      // S^T_{i+1} overwrites P^T_i in A: issued after dV_i (same thread, in
+      // order) and after the softmax finished reading P^T_i (ds_full).
+      // dP^T_{i+1} overwrites dS^T_i in B: issued after dK_i, in order.
+      bool ok = mbar_wait(kv_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int st = it & 1;
+        const uint32_t q_addr = sbase + C::Q_OFF + st * C::TILE;
+        const uint32_t do_addr = sbase + C::DO_OFF + st * C::TILE;
+        // dV += P^T dO_i: query k-step kk (16 queries) lives in columns
+        // 64*(kk/4) + 8*(kk%4) of region A.
         if (!mbar_wait(p_full, it & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + kColDV, tmem + kColS + kk * 8,
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_ts(tmem + kKvColDV, tmem + kKvColS + (kk >> 2) * 64 + (kk & 3) * 8,
                  sdesc_sw128(do_addr + kk * 2048, C::BLK, 1024), kIdescAcc,
                  (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q_i and dQ_i = dS K_j (into the dP^T columns).
         if (!mbar_wait(ds_full, it & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
+        if (it + 1 < n_iter && !issue_s(it + 1)) break;
+        // dK += dS^T Q_i: dS^T k-step kk at column 128 + 64*(kk/4) + 8*(kk%4).
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + off, 16, 1024),
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_ts(tmem + kKvColDK, tmem + kKvColDP + (kk >> 2) * 64 + (kk & 3) * 8,
                  sdesc_sw128(q_addr + kk * 2048, C::BLK, 1024), kIdescAcc,
                  (it > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_ss(tmem + kColDP, sdesc_sw128(ds_addr + kk * 2048, C::BLK, 1024),
-                 sdesc_sw128(k_addr + kk * 2048, C::BLK, 1024), kIdescDq, kk > 0 ? 1u : 0u);
-        mma_commit(dq_full);
         mma_commit(qdo_empty + st);
-        // S^T of the next query tile overlaps the dQ readout.
-        if (it + 1 < n_iter) ok = issue_s(it + 1);
+        if (it + 1 < n_iter && !issue_dp(it + 1)) break;
       }
       mma_commit(kv_done);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------- P^T and dS^T (warps 0..3)
-    const int kr = threadIdx.x;  // key row == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int k_idx = j * kBM + kr;
+  } else {
+    // ------------------------- P^T and dS^T (warps 0-3: queries 0-63, 4-7: 64-127)
+    const int h = warp >> 2;
+    const int kr = threadIdx.x & 127;  // key row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t col_s = kKvColS + 64 * h;    // this half's S^T, then P^T
+    const uint32_t col_dp = kKvColDP + 64 * h;  // this half's dP^T, then dS^T
+    const int k_idx = j * kT + kr;
     const bool key_ok = k_idx < N;
-    uint8_t* ds_tile = smem + C::DS_OFF;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int i = i_start + it;
-      const float* l2 = lse2 + static_cast<size_t>(bh) * Np + i * kBN;
-      const float* dd = dvec + static_cast<size_t>(bh) * Np + i * kBN;
+      const int st = it & 1;
+      // LSE2 and D of this half's 64 queries, staged by the producer with
+      // the Q tile (q_full[st] completed before S^T, hence before s_full).
+      const float* l2 = reinterpret_cast<const float*>(smem + C::VEC_OFF + st * 1024) + 64 * h;
+      const float* dd = l2 + 128;
       const bool diag = CAUSAL && (i == j);
       if (!wait_all(s_full, it & 1, abort, ctl, kSiteBwdSoftmax)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      uint32_t sv[2][32];
+      tmem_ld32(lane_base + col_s, sv[0]);
+      tmem_ld32(lane_base + col_s + 32, sv[1]);
+      tmem_wait_ld();
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      // queries of this half this key row sees: all, none (key past N), or
+      // q >= key on the diagonal tile
+      const int qlo = !key_ok ? 64 : (diag ? kr - 64 * h : 0);
+      uint32_t pk[32];  // P^T of this half, bf16 pairs
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(lane_base + kColS + c * 32, sv);
-        tmem_wait_ld();
-        uint32_t pk[16];
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float4 lv = __ldg(reinterpret_cast<const float4*>(l2 + c * 32 + e));
-          float p[4];
-          p[0] = ex2(fmaf(__uint_as_float(sv[e + 0]), scale_log2, -lv.x));
-          p[1] = ex2(fmaf(__uint_as_float(sv[e + 1]), scale_log2, -lv.y));
-          p[2] = ex2(fmaf(__uint_as_float(sv[e + 2]), scale_log2, -lv.z));
-          p[3] = ex2(fmaf(__uint_as_float(sv[e + 3]), scale_log2, -lv.w));
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int qcol = c * 32 + e + t;
-            if (!key_ok || (diag && qcol < kr)) p[t] = 0.f;
-          }
-          pk[e / 2] = pack_bf16(p[0], p[1]);
-          pk[e / 2 + 1] = pack_bf16(p[2], p[3]);
+          const float4 lv = *reinterpret_cast<const float4*>(l2 + c * 32 + e);
+          const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e]),
+                                                    __uint_as_float(sv[c][e + 1])),
+                                        sc2, make_float2(-lv.x, -lv.y));
+          const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e + 2]),
+                                                    __uint_as_float(sv[c][e + 3])),
+                                        sc2, make_float2(-lv.z, -lv.w));
+          // one pair in three on the FMA pipe, the rest on the MUFU
+          float2 p01, p23;
+          if (((c * 16 + e / 2) % 3) == 2)
+            p01 = exp2_fma2(x01);
+          else
+            p01 = make_float2(ex2(x01.x), ex2(x01.y));
+          if (((c * 16 + e / 2 + 1) % 3) == 2)
+            p23 = exp2_fma2(x23);
+          else
+            p23 = make_float2(ex2(x23.x), ex2(x23.y));
+          const int q0 = c * 32 + e;  // query within this half
+          if (q0 + 0 < qlo) p01.x = 0.f;
+          if (q0 + 1 < qlo) p01.y = 0.f;
+          if (q0 + 2 < qlo) p23.x = 0.f;
+          if (q0 + 3 < qlo) p23.y = 0.f;
+          pk[c * 16 + e / 2] = pack_bf16(p01.x, p01.y);
+          pk[c * 16 + e / 2 + 1] = pack_bf16(p23.x, p23.y);
         }
-        // P^T columns [16c, 16c+16) lie in S^T columns already read.
-        tmem_st16(lane_base + kColS + c * 16, pk);
       }
+      // P^T -> columns [col_s, col_s + 32): already read above.
+      tmem_st32(lane_base + col_s, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
 
-      // dS^T needs the dS buffer back (dK/dQ MMAs and the dQ staging of
-      // iteration it-1 are done with it) and dP^T of this iteration.
-      if (it > 0 && !wait_all(ds_free, (it - 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
-        ok = false;
-        break;
-      }
       if (!wait_all(dp_full, it & 1, abort, ctl, kSiteBwdSoftmax)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      uint32_t dpv[2][32];
+      tmem_ld32(lane_base + col_dp, dpv[0]);
+      tmem_ld32(lane_base + col_dp + 32, dpv[1]);
+      tmem_wait_ld();
+      uint32_t dsk[32];
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t dpv[32], pk[16];
-        tmem_ld32(lane_base + kColDP + c * 32, dpv);
-        tmem_ld16(lane_base + kColS + c * 16, pk);
-        tmem_wait_ld();
-        uint32_t dsk[16];
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float4 dv4 = __ldg(reinterpret_cast<const float4*>(dd + c * 32 + e));
-          const float d0 = bf16lo(pk[e / 2]) * (__uint_as_float(dpv[e + 0]) - dv4.x);
-          const float d1 = bf16hi(pk[e / 2]) * (__uint_as_float(dpv[e + 1]) - dv4.y);
-          const float d2 = bf16lo(pk[e / 2 + 1]) * (__uint_as_float(dpv[e + 2]) - dv4.z);
-          const float d3 = bf16hi(pk[e / 2 + 1]) * (__uint_as_float(dpv[e + 3]) - dv4.w);
-          dsk[e / 2] = pack_bf16(d0, d1);
-          dsk[e / 2 + 1] = pack_bf16(d2, d3);
+          const float4 dv4 = *reinterpret_cast<const float4*>(dd + c * 32 + e);
+          const uint32_t p01 = pk[c * 16 + e / 2], p23 = pk[c * 16 + e / 2 + 1];
+          const float d0 = bf16lo(p01) * (__uint_as_float(dpv[c][e + 0]) - dv4.x);
+          const float d1 = bf16hi(p01) * (__uint_as_float(dpv[c][e + 1]) - dv4.y);
+          const float d2 = bf16lo(p23) * (__uint_as_float(dpv[c][e + 2]) - dv4.z);
+          const float d3 = bf16hi(p23) * (__uint_as_float(dpv[c][e + 3]) - dv4.w);
+          dsk[c * 16 + e / 2] = pack_bf16(d0, d1);
+          dsk[c * 16 + e / 2 + 1] = pack_bf16(d2, d3);
         }
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-          st_sw128(ds_tile, kr, c * 4 + h,
-                   make_uint4(dsk[4 * h], dsk[4 * h + 1], dsk[4 * h + 2], dsk[4 * h + 3]));
       }
-      fence_async_shared();
+      // dS^T -> columns [col_dp, col_dp + 32): dP^T values there were read.
+      tmem_st32(lane_base + col_dp, dsk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(ds_full);
     }
-    // dV epilogue
+    // Epilogue: dV (unscaled) and dK (times scale), 16-column steps split
+    // between the two warpgroups.
     if (ok && wait_all(kv_done, 0, abort, ctl, kSiteBwdEpilogue)) {
       tc_fence_after();
-      uint4* row = reinterpret_cast<uint4*>(dv + (static_cast<size_t>(bh) * N + k_idx) * D);
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t v16[16];
-        tmem_ld16(lane_base + kColDV + c * 16, v16);
-        tmem_wait_ld();
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          pk[e] = pack_bf16(__uint_as_float(v16[2 * e]), __uint_as_float(v16[2 * e + 1]));
-        if (key_ok) {
-          row[2 * c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          row[2 * c + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-      }
-    }
-  } else {
-    // --------------------------------------------- dQ readout (warps 4..7)
-    const int wq = warp - 4;           // TMEM lane quarter: query rows 32*wq..
-    const int qr = threadIdx.x - 128;  // query row == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    // Per-warp staging: two 32 x 32 fp32 sub-tiles (4 KB each, 128-byte
-    // swizzled) inside the dS buffer.
-    uint8_t* stage = smem + C::DS_OFF + wq * 8192;
-    bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      const int q0 = (i_start + it) * kBN;
-      if (!wait_all(dq_full, it & 1, abort, ctl, kSiteBwdDq)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int pass = 0; pass < (C::NSUB + 1) / 2; ++pass) {
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          const int sub = 2 * pass + sl;
-          if (sub < C::NSUB) {
-            uint32_t v[32];
-            tmem_ld32(lane_base + kColDP + sub * 32, v);
-            tmem_wait_ld();
-            uint8_t* rowp = stage + sl * 4096 + lane * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float4 f = make_float4(__uint_as_float(v[4 * c]) * scale,
-                                           __uint_as_float(v[4 * c + 1]) * scale,
-                                           __uint_as_float(v[4 * c + 2]) * scale,
-                                           __uint_as_float(v[4 * c + 3]) * scale);
-              *reinterpret_cast<float4*>(rowp + ((c ^ (lane & 7)) * 16)) = f;
-            }
-          }
-        }
-        if (2 * pass + 2 >= C::NSUB) {
-          // Last TMEM read of dQ_i: release the dP^T columns.
-          tc_fence_before();
-          mbar_arrive(dq_empty);
-        }
-        fence_async_shared();
-        __syncwarp();
-        if (lane == 0) {
-          const int y = q0 + wq * 32;
-          if (y < N) {
-#pragma unroll
-            for (int sl = 0; sl < 2; ++sl)
-              if (2 * pass + sl < C::NSUB)
-                tma_reduce_add_3d(&tm_dq, stage + sl * 4096, (2 * pass + sl) * 32, y, bh);
-          }
-          bulk_commit();
-          bulk_wait_read_all();
-        }
-        __syncwarp();
-      }
-      if (lane == 0) mbar_arrive(ds_free);
-      (void)qr;
-    }
-    if (lane == 0) bulk_wait_all();
-    __syncwarp();
-    // dK epilogue
-    if (ok && wait_all(kv_done, 0, abort, ctl, kSiteBwdEpilogue)) {
-      tc_fence_after();
-      const int k_idx = j * kBM + qr;
-      uint4* row = reinterpret_cast<uint4*>(dk + (static_cast<size_t>(bh) * N + k_idx) * D);
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t v16[16];
-        tmem_ld16(lane_base + kColDK + c * 16, v16);
-        tmem_wait_ld();
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          pk[e] = pack_bf16(__uint_as_float(v16[2 * e]) * scale,
-                            __uint_as_float(v16[2 * e + 1]) * scale);
-        if (k_idx < N) {
-          row[2 * c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          row[2 * c + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-      }
+      const size_t row = (static_cast<size_t>(bh) * N + k_idx) * D;
+      store_row_bf16<D>(lane_base + kKvColDV, 1.f, dv + row, key_ok, h);
+      store_row_bf16<D>(lane_base + kKvColDK, scale, dk + row, key_ok, h);
     }
   }
 
@@ -480,45 +430,325 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// =========================================================================
+// dQ
+// =========================================================================
+
+template <int D>
+struct QCfg : Shape<D> {
+  using S = Shape<D>;
+  // K_j is used by S_j and dQ_j (late), V_j only by dP_j (early), so the K
+  // ring is one stage deeper: K_{j+2} can land while dQ_j still reads K_j.
+  static constexpr int NK = S::NB == 1 ? 4 : 3;
+  static constexpr int NV = S::NB == 1 ? 4 : 2;
+  static constexpr int Q_OFF = 0;
+  static constexpr int DO_OFF = Q_OFF + S::TILE;
+  static constexpr int K_OFF = DO_OFF + S::TILE;      // [NK]
+  static constexpr int V_OFF = K_OFF + NK * S::TILE;  // [NV]
+  static constexpr int BAR_OFF = V_OFF + NV * S::TILE;
+  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 5;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// TMEM columns of the dQ kernel: S double buffer, dP, dQ accumulator.
+// Softmax warpgroup h reads S columns [64h, 64h+64) of the current buffer and
+// writes its dS (bf16 pairs) into [64h, 64h+32) of the same buffer.
+constexpr uint32_t kQColS = 0, kQColDP = 256, kQColDQ = 384;
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ dvec,
+                  const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dq, int N, int BH,
+                  int group, float scale, float scale_log2, WaitCtl ctl) {
+  using C = QCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* q_full = bars + 0;  // Q_i and dO_i
+  uint64_t* dq_done = bars + 1;
+  uint64_t* k_full = bars + 2;          // [NK]
+  uint64_t* k_empty = k_full + C::NK;   // [NK]
+  uint64_t* v_full = k_empty + C::NK;   // [NV]
+  uint64_t* v_empty = v_full + C::NV;   // [NV]
+  uint64_t* s_full = v_empty + C::NV;   // [2] per S buffer
+  uint64_t* ds_full = s_full + 2;         // [2] per S buffer
+  uint64_t* dp_full = ds_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int n_t = (N + kT - 1) / kT;
+  const int Np = n_t * kT;
+  int bh, t;
+  group_major(n_t, BH, group, bh, t);
+  const int i = n_t - 1 - t;  // longest query tiles first when causal
+  const int n_kv = CAUSAL ? i + 1 : n_t;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(dq_done, 1);
+    for (int s = 0; s < C::NK; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < C::NV; ++s) {
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(ds_full + b, 2 * kT);
+    }
+    mbar_init(dp_full, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      int last_k[C::NK], last_v[C::NV];
+#pragma unroll
+      for (int s = 0; s < C::NK; ++s) last_k[s] = -1;
+#pragma unroll
+      for (int s = 0; s < C::NV; ++s) last_v[s] = -1;
+      mbar_arrive_expect_tx(q_full, 2 * C::TILE);
+#pragma unroll
+      for (int b = 0; b < C::NB; ++b) {
+        tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + b * C::BLK, b * 64, i * kT, bh);
+        tma_load_3d(&tm_do, q_full, smem + C::DO_OFF + b * C::BLK, b * 64, i * kT, bh);
+      }
+      for (int jj = 0; jj < n_kv; ++jj) {
+        const int sk = jj % C::NK, sv = jj % C::NV;
+        const uint32_t uk = static_cast<uint32_t>(jj / C::NK);
+        const uint32_t uv = static_cast<uint32_t>(jj / C::NV);
+        if (jj >= C::NK && !mbar_wait(k_empty + sk, (uk - 1) & 1, abort, ctl, kSiteBwdProducer))
+          break;
+        mbar_arrive_expect_tx(k_full + sk, C::TILE);
+#pragma unroll
+        for (int b = 0; b < C::NB; ++b)
+          tma_load_3d(&tm_k, k_full + sk, smem + C::K_OFF + sk * C::TILE + b * C::BLK, b * 64,
+                      jj * kT, bh);
+        last_k[sk] = static_cast<int>(uk);
+        if (jj >= C::NV && !mbar_wait(v_empty + sv, (uv - 1) & 1, abort, ctl, kSiteBwdProducer))
+          break;
+        mbar_arrive_expect_tx(v_full + sv, C::TILE);
+#pragma unroll
+        for (int b = 0; b < C::NB; ++b)
+          tma_load_3d(&tm_v, v_full + sv, smem + C::V_OFF + sv * C::TILE + b * C::BLK, b * 64,
+                      jj * kT, bh);
+        last_v[sv] = static_cast<int>(uv);
+      }
+      if (*abort) {
+        drain_wait(q_full, 0, ctl);
+        for (int s = 0; s < C::NK; ++s)
+          if (last_k[s] >= 0) drain_wait(k_full + s, last_k[s] & 1, ctl);
+        for (int s = 0; s < C::NV; ++s)
+          if (last_v[s] >= 0) drain_wait(v_full + s, last_v[s] & 1, ctl);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S, dP
+      constexpr uint32_t kIdescDq = idesc_bf16(kT, D, 0, 1);   // dQ (B = K_j MN-major)
+      const uint32_t q_addr = sbase + C::Q_OFF;
+      const uint32_t do_addr = sbase + C::DO_OFF;
+      auto issue_s = [&](int jj) -> bool {  // S_jj = Q K_jj^T -> buffer jj % 2
+        const int s = jj % C::NK;
+        if (!mbar_wait(k_full + s, (jj / C::NK) & 1, abort, ctl, kSiteBwdMma)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = sbase + C::K_OFF + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          mma_ss(tmem + kQColS + (jj & 1) * kT, sdesc_sw128(q_addr + off, 16, 1024),
+                 sdesc_sw128(k_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full + (jj & 1));
+        return true;
+      };
+      auto issue_dp = [&](int jj) -> bool {  // dP_jj = dO V_jj^T, then V_jj is free
+        const int s = jj % C::NV;
+        if (!mbar_wait(v_full + s, (jj / C::NV) & 1, abort, ctl, kSiteBwdMma)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = sbase + C::V_OFF + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          mma_ss(tmem + kQColDP, sdesc_sw128(do_addr + off, 16, 1024),
+                 sdesc_sw128(v_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(dp_full);
+        mma_commit(v_empty + s);
+        return true;
+      };
+      // Order: S_0, dP_0, S_1, [dS_0] dQ_0, dP_1, S_2, [dS_1] dQ_1, ... so the
+      // tensor core computes S_{j+1} while the softmax warps form dS_j.  S_{j+2}
+      // reuses S_j's buffer after dQ_j has read dS_j (same thread, in order)
+      // and the softmax released it (ds_full waited); dP_{j+1} likewise.
+      bool ok = mbar_wait(q_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
+      if (ok && n_kv > 1) ok = issue_s(1);
+      for (int jj = 0; ok && jj < n_kv; ++jj) {
+        const int s = jj % C::NK;
+        if (!mbar_wait(ds_full + (jj & 1), (jj >> 1) & 1, abort, ctl, kSiteBwdMma)) break;
+        tc_fence_after();
+        const uint32_t k_addr = sbase + C::K_OFF + s * C::TILE;
+        // dQ += dS_jj K_jj: key k-step kk (16 keys) of dS at column
+        // 64*(kk/4) + 8*(kk%4) of the S buffer.
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_ts(tmem + kQColDQ, tmem + kQColS + (jj & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
+                 sdesc_sw128(k_addr + kk * 2048, C::BLK, 1024), kIdescDq,
+                 (jj > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(k_empty + s);
+        if (jj + 1 < n_kv && !issue_dp(jj + 1)) break;
+        if (jj + 2 < n_kv && !issue_s(jj + 2)) break;
+      }
+      mma_commit(dq_done);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------- dS (warps 0-3: keys 0-63, 4-7: keys 64-127)
+    const int h = warp >> 2;
+    const int qr = threadIdx.x & 127;  // query row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int q_idx = i * kT + qr;
+    const float my_l2 = lse2[static_cast<size_t>(bh) * Np + q_idx];  // +inf past N
+    const float my_d = dvec[static_cast<size_t>(bh) * Np + q_idx];
+    bool ok = true;
+    for (int jj = 0; jj < n_kv; ++jj) {
+      const uint32_t col_s = kQColS + (jj & 1) * kT + 64 * h;
+      if (!wait_all(s_full + (jj & 1), (jj >> 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[2][32];
+      tmem_ld32(lane_base + col_s, sv[0]);
+      tmem_ld32(lane_base + col_s + 32, sv[1]);
+      tmem_wait_ld();
+      const int k0 = jj * kT + 64 * h;  // first key of this half
+      // keys k visible to this query: k <= q_idx (causal) and k < N
+      const int lim = min(N, CAUSAL ? q_idx + 1 : N) - k0;
+      float p[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float x = fmaf(__uint_as_float(sv[c >> 5][c & 31]), scale_log2, -my_l2);
+        p[c] = (c < lim) ? ex2(x) : 0.f;
+      }
+      if (!wait_all(dp_full, jj & 1, abort, ctl, kSiteBwdSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t dpv[2][32];
+      tmem_ld32(lane_base + kQColDP + 64 * h, dpv[0]);
+      tmem_ld32(lane_base + kQColDP + 64 * h + 32, dpv[1]);
+      tmem_wait_ld();
+      uint32_t dsk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int c0 = 2 * c, c1 = 2 * c + 1;
+        const float d0 = p[c0] * (__uint_as_float(dpv[c0 >> 5][c0 & 31]) - my_d);
+        const float d1 = p[c1] * (__uint_as_float(dpv[c1 >> 5][c1 & 31]) - my_d);
+        dsk[c] = pack_bf16(d0, d1);
+      }
+      // dS -> columns [col_s, col_s + 32) of the S buffer (already read).
+      tmem_st32(lane_base + col_s, dsk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full + (jj & 1));
+    }
+    if (ok && wait_all(dq_done, 0, abort, ctl, kSiteBwdEpilogue)) {
+      tc_fence_after();
+      store_row_bf16<D>(lane_base + kQColDQ, scale, dq + (static_cast<size_t>(bh) * N + q_idx) * D,
+                        q_idx < N, h);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ launch
+
+inline int heads_per_group(long long per_head_bytes, int BH) {
+  int g = static_cast<int>((48LL << 20) / (per_head_bytes > 0 ? per_head_bytes : 1));
+  return g < 1 ? 1 : (g > BH ? BH : g);
+}
+
 template <int D, bool CAUSAL>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const CUtensorMap& tdo, const CUtensorMap& tdq, const float* dvec,
-                   const float* lse2, void* dk, void* dv, int BH, int N, float scale,
-                   const Launch& L) {
-  using C = Cfg<D>;
+                   const CUtensorMap& tdo, const float* dvec, const float* lse2, void* dq,
+                   void* dk, void* dv, int BH, int N, float scale, const Launch& L) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_kernel<D, CAUSAL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, CAUSAL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         KvCfg<D>::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D, CAUSAL>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, QCfg<D>::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int n_kv = (N + kBM - 1) / kBM;
-  // Heads per group: keep a group's K, V, Q, dO (bf16) and dQ accumulator
-  // (fp32), 12 N d bytes per head, within ~48 MB of the 126 MB L2.
-  const long long per_head = 12LL * N * D;
-  int group = static_cast<int>((48LL << 20) / (per_head > 0 ? per_head : 1));
-  group = group < 1 ? 1 : (group > BH ? BH : group);
-  const long long blocks = static_cast<long long>(BH) * n_kv;
+  const int n_t = (N + kT - 1) / kT;
+  const long long blocks = static_cast<long long>(BH) * n_t;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  // Heads per group: a group's Q, K, V, dO (bf16, 8 N d bytes per head)
+  // within ~48 MB of the 126 MB L2.
+  const int group = heads_per_group(8LL * N * D, BH);
+  const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};
-  bwd_kernel<D, CAUSAL><<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
-      tq, tk, tv, tdo, tdq, dvec, lse2, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), N, BH, group, scale, scale * 1.4426950408889634f, ctl);
+  bwd_dkdv_kernel<D, CAUSAL>
+      <<<static_cast<unsigned>(blocks), kThreads, KvCfg<D>::SMEM, L.stream>>>(
+          tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dk),
+          static_cast<__nv_bfloat16*>(dv), N, BH, group, scale, scale_log2, ctl);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dq_kernel<D, CAUSAL><<<static_cast<unsigned>(blocks), kThreads, QCfg<D>::SMEM, L.stream>>>(
+      tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dq), N, BH, group, scale,
+      scale_log2, ctl);
   return cudaGetLastError();
 }
 
 }  // namespace bwd
 
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tdo, const CUtensorMap& tdq, const float* dvec,
-                             const float* lse2, void* dk, void* dv, int BH, int N, int d,
-                             float scale, int causal, const Launch& L) {
-#define FA_BWD_CASE(DD)                                                                     \
-  case DD:                                                                                  \
-    return causal ? bwd::launch<DD, true>(tq, tk, tv, tdo, tdq, dvec, lse2, dk, dv, BH, N,  \
-                                          scale, L)                                         \
-                  : bwd::launch<DD, false>(tq, tk, tv, tdo, tdq, dvec, lse2, dk, dv, BH, N, \
+                             const CUtensorMap& tdo, const float* dvec, const float* lse2,
+                             void* dq, void* dk, void* dv, int BH, int N, int d, float scale,
+                             int causal, const Launch& L) {
+#define FA_BWD_CASE(DD)                                                                       \
+  case DD:                                                                                    \
+    return causal ? bwd::launch<DD, true>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N,     \
+                                          scale, L)                                           \
+                  : bwd::launch<DD, false>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N,    \
                                            scale, L);
   switch (d) {
     FA_BWD_CASE(64)

@@ -11,19 +11,25 @@
 // P never leave the SM: S lives in tensor memory (TMEM), P is written back
 // over S as bf16 and fed to the second MMA straight from TMEM.
 //
-// B200 design (one CTA per 128-row query tile, 6 warps):
-//   warp 4      TMA producer: Q tile once, then K_j and V_j into separate
-//               3- or 4-stage shared-memory rings (mbarrier full/empty pairs).
-//   warp 5      TMEM allocator and single-thread MMA issuer:
-//               S_j = Q K_j^T into TMEM buffer j%2 (SS form), then
-//               O += P_{j-1} V_{j-1} with P read from TMEM (TS form), so the
-//               tensor core computes S_j while the softmax works on S_{j-1}.
-//   warps 0-3   softmax: one thread per query row (= TMEM lane).  Base-2
-//               domain, lazy rescaling: the reference max is only moved
-//               (and O, l rescaled in TMEM) when the row max grew by more
-//               than 2^8, which keeps every exponent <= 8 and makes O
-//               corrections rare after the first tiles.  They also run the
-//               epilogue (O / l -> bf16, LSE).
+// B200 design: one CTA per pair of 128-row query tiles (A = 2p, B = 2p+1)
+// of one head, 12 warps (warps 10-11 idle; the third warpgroup gives its
+// registers to the two softmax warpgroups):
+//   warp 8      TMA producer: both Q tiles once, then K_j and V_j into
+//               separate shared-memory rings; each K/V tile serves both Q
+//               tiles (half the K/V traffic per FLOP of a one-tile CTA).
+//   warp 9      TMEM allocator and single-thread MMA issuer, alternating
+//               between the tiles: O_A += P_A V_j, S_A = Q_A K_{j+1}^T,
+//               O_B += P_B V_j, S_B = Q_B K_{j+1}^T, so the tensor core works
+//               on one tile while the other tile's softmax runs.
+//   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: one thread
+//               per query row (= TMEM lane), base-2 domain, lazy rescaling
+//               (the reference max moves, and O and l are rescaled in TMEM,
+//               only when the row max grew by more than 2^8; exponents stay
+//               <= 8).  They also run their tile's epilogue (O / l, LSE).
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+d),
+// O_B [384,384+d).  S of a tile is single-buffered: S_X(j+1) is issued after
+// O_X += P_X(j) V_j, so when the softmax sees S_X(j+1) the previous P V has
+// completed and O_X can be rescaled without waiting.
 // Causal: tiles above the diagonal are never loaded; only the diagonal tile
 // and a ragged last tile are masked.  CTAs run group-major (a few heads at a
 // time, so their K and V stay in L2), longest-first inside a group.
@@ -37,22 +43,26 @@ namespace fwd {
 
 constexpr int kBM = 128;              // query rows per tile (TMEM lanes)
 constexpr int kBN = 128;              // keys per K/V tile
-constexpr int kThreads = 192;         // 4 softmax warps + producer + MMA
+constexpr int kThreads = 384;         // 2 softmax warpgroups + producer/MMA warpgroup
+// Registers per thread: 168 at launch (384 threads), then the softmax
+// warpgroups take 224 and the producer/MMA warpgroup keeps 56:
+// 224 + 224 + 56 = 504 = 3 x 168, the launch budget of each lane slot.
+constexpr int kLaunchRegs = 168, kSoftmaxRegs = 224, kControlRegs = 56;
+static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kLaunchRegs, "register split over budget");
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;       // O accumulator columns [256, 256+d)
 
 template <int D>
 struct Cfg {
   static constexpr int NB = (D + 63) / 64;  // 64-column (128-byte) swizzle blocks
   static constexpr int BLK = 64 * kBM * 2;  // bytes of one 128 x 64 bf16 block
   static constexpr int TILE = NB * BLK;     // bytes of one Q/K/V tile
-  static constexpr int NST = NB == 1 ? 4 : 3;
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + TILE;
+  static constexpr int NST = NB == 1 ? 4 : 2;
+  static constexpr int Q_OFF = 0;           // [2] tiles A, B
+  static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + NST * TILE;
   static constexpr int BAR_OFF = V_OFF + NST * TILE;
-  static constexpr int NBAR = 1 + 4 * NST + 2 + 2 + 1;
+  static constexpr int NBAR = 1 + 4 * NST + 6;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;  // + slack for 1 KB alignment
   static constexpr int KSTEPS = D / 16;
@@ -70,6 +80,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const
       return;
     }
   }
+}
+
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                         const WaitCtl& ctl, int site) {
+  const bool w = mbar_wait(bar, parity, abort, ctl, site);
+  return __all_sync(0xffffffffu, w);
 }
 
 template <int D, bool CAUSAL>
@@ -90,28 +106,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = k_full + C::NST;
   uint64_t* v_full = k_empty + C::NST;
   uint64_t* v_empty = v_full + C::NST;
-  uint64_t* s_full = v_empty + C::NST;  // [2]
-  uint64_t* p_full = s_full + 2;        // [2]
-  uint64_t* o_done = p_full + 2;
+  uint64_t* s_full = v_empty + C::NST;  // [2] per tile
+  uint64_t* p_full = s_full + 2;        // [2] per tile
+  uint64_t* o_done = p_full + 2;        // [2] per tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int n_kv_all = (N + kBN - 1) / kBN;
+  const int n_t = (N + kBN - 1) / kBN;  // query tiles == key tiles
+  const int n_pair = (n_t + 1) / 2;
   // Group-major order: `group` heads at a time (their K and V stay in L2),
-  // and inside a group the longest query tiles first, head fastest.
-  int bh, qt;
+  // and inside a group the longest tile pairs first, head fastest.
+  int bh, pair;
   {
-    const int per_group = group * n_kv_all;
+    const int per_group = group * n_pair;
     const int g = static_cast<int>(blockIdx.x) / per_group;
     const int r = static_cast<int>(blockIdx.x) - g * per_group;
     const int gh = min(group, BH - g * group);
     const int t = r / gh;
-    qt = n_kv_all - 1 - t;
+    pair = n_pair - 1 - t;
     bh = g * group + (r - t * gh);
   }
-  const int n_kv = CAUSAL ? min(qt + 1, n_kv_all) : n_kv_all;
+  const int qt[2] = {2 * pair, 2 * pair + 1};
+  // Key tiles each query tile visits (0 when tile B lies past N).
+  int n_x[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x)
+    n_x[x] = qt[x] >= n_t ? 0 : (CAUSAL ? min(qt[x] + 1, n_t) : n_t);
+  const int n_max = max(n_x[0], n_x[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -121,15 +144,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(v_full + s, 1);
       mbar_init(v_empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full + b, 1);
-      mbar_init(p_full + b, kBM);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_full + x, kBM);
+      mbar_init(o_done + x, 1);
     }
-    mbar_init(o_done, 1);
     *abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -138,7 +161,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp >= 8) {
+  regs_decrease<kControlRegs>();
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -147,11 +172,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last_k[C::NST], last_v[C::NST];
 #pragma unroll
       for (int s = 0; s < C::NST; ++s) last_k[s] = last_v[s] = -1;
-      mbar_arrive_expect_tx(q_full, C::TILE);
+      const int nq = n_x[1] > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, nq * C::TILE);
+      for (int x = 0; x < nq; ++x)
 #pragma unroll
-      for (int b = 0; b < C::NB; ++b)
-        tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + b * C::BLK, b * 64, qt * kBM, bh);
-      for (int j = 0; j < n_kv; ++j) {
+        for (int b = 0; b < C::NB; ++b)
+          tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + x * C::TILE + b * C::BLK, b * 64,
+                      qt[x] * kBM, bh);
+      for (int j = 0; j < n_max; ++j) {
         const int s = j % C::NST;
         const uint32_t u = static_cast<uint32_t>(j / C::NST);
         if (j >= C::NST && !mbar_wait(k_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer))
@@ -181,66 +209,88 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, 0, 0);
       constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, 0, 1);
-      const uint32_t q_addr = sbase + C::Q_OFF;
-      auto issue_pv = [&](int t) -> bool {
-        const int sb = t & 1;
-        if (!mbar_wait(p_full + sb, (t >> 1) & 1, abort, ctl, kSiteFwdMma)) return false;
-        const int s = t % C::NST;
-        if (!mbar_wait(v_full + s, (t / C::NST) & 1, abort, ctl, kSiteFwdMma)) return false;
+      int k_seen = -1;  // highest key tile whose k_full wait has been done
+      auto wait_k = [&](int jj) -> bool {
+        if (jj <= k_seen) return true;
+        if (!mbar_wait(k_full + jj % C::NST, (jj / C::NST) & 1, abort, ctl, kSiteFwdMma))
+          return false;
+        k_seen = jj;
         tc_fence_after();
-        const uint32_t v_addr = sbase + C::V_OFF + s * C::TILE;
-        const uint32_t p_tmem = tmem + sb * kBN;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // V_j as the K x N (keys x d) operand, d contiguous: MN-major.
-          const uint64_t bdesc = sdesc_sw128(v_addr + kk * 16 * 128, C::BLK, 1024);
-          mma_ts(tmem + kColO, p_tmem + kk * 8, bdesc, kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(v_empty + s);
-        mma_commit(o_done);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, abort, ctl, kSiteFwdMma);
-      tc_fence_after();
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % C::NST;
-        if (!mbar_wait(k_full + s, (j / C::NST) & 1, abort, ctl, kSiteFwdMma)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_addr = sbase + C::K_OFF + s * C::TILE;
-        const uint32_t s_tmem = tmem + (j & 1) * kBN;
+      auto issue_s = [&](int x, int jj) {  // S_x = Q_x K_jj^T
+        const uint32_t q_addr = sbase + C::Q_OFF + x * C::TILE;
+        const uint32_t k_addr = sbase + C::K_OFF + (jj % C::NST) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(s_tmem, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                 kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + x * kBN, sdesc_sw128(q_addr + off, 16, 1024),
+                 sdesc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full + (j & 1));
-        mma_commit(k_empty + s);
-        if (j > 0) ok = issue_pv(j - 1);
+        mma_commit(s_full + x);
+      };
+      auto issue_pv = [&](int x, int jj) {  // O_x += P_x V_jj, P_x from TMEM
+        const uint32_t v_addr = sbase + C::V_OFF + (jj % C::NST) * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(tmem + 256 + x * kBN, tmem + x * kBN + kk * 8,
+                 sdesc_sw128(v_addr + kk * 16 * 128, C::BLK, 1024), kIdescPV,
+                 (jj > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(o_done + x);
+      };
+      bool ok = mbar_wait(q_full, 0, abort, ctl, kSiteFwdMma) && wait_k(0);
+      if (ok) {
+        tc_fence_after();
+        for (int x = 0; x < 2; ++x)
+          if (n_x[x] > 0) issue_s(x, 0);
+        mma_commit(k_empty + 0);
       }
-      if (ok) issue_pv(n_kv - 1);
+      for (int j = 0; ok && j < n_max; ++j) {
+        const int s = j % C::NST;
+        if (!mbar_wait(v_full + s, (j / C::NST) & 1, abort, ctl, kSiteFwdMma)) break;
+        for (int x = 0; ok && x < 2; ++x) {
+          if (j >= n_x[x]) continue;
+          if (!mbar_wait(p_full + x, j & 1, abort, ctl, kSiteFwdMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(x, j);
+          if (j + 1 < n_x[x]) {
+            if (!wait_k(j + 1)) {
+              ok = false;
+              break;
+            }
+            issue_s(x, j + 1);
+          }
+        }
+        if (!ok) break;
+        mma_commit(v_empty + s);
+        if (j + 1 < n_max) mma_commit(k_empty + (j + 1) % C::NST);
+      }
     }
     __syncwarp();
+  }
   } else {
-    // ------------------------------------------------ softmax (warps 0..3)
-    const int r = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int q_idx = qt * kBM + r;
+    regs_increase<kSoftmaxRegs>();
+    // --------------------------------------- softmax (warps 0-3: A, 4-7: B)
+    const int x = warp >> 2;
+    const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t col_s = x * kBN;
+    const uint32_t col_o = 256 + x * kBN;
+    const int n_kv = n_x[x];
+    const int q_idx = qt[x] * kBM + r;
     float m = -INFINITY;  // reference max, base-2 scaled units
     float l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      const bool w = mbar_wait(s_full + sb, (j >> 1) & 1, abort, ctl, kSiteFwdSoftmax);
-      if (!__all_sync(0xffffffffu, w)) {
+      if (!wait_all(s_full + x, j & 1, abort, ctl, kSiteFwdSoftmax)) {
         ok = false;
         break;
       }
@@ -248,16 +298,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       float s[kBN];
       {
         uint32_t t0[32], t1[32];
-        tmem_ld32(lane_base + sb * kBN + 0, t0);
-        tmem_ld32(lane_base + sb * kBN + 32, t1);
+        tmem_ld32(lane_base + col_s + 0, t0);
+        tmem_ld32(lane_base + col_s + 32, t1);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           s[c] = __uint_as_float(t0[c]);
           s[32 + c] = __uint_as_float(t1[c]);
         }
-        tmem_ld32(lane_base + sb * kBN + 64, t0);
-        tmem_ld32(lane_base + sb * kBN + 96, t1);
+        tmem_ld32(lane_base + col_s + 64, t0);
+        tmem_ld32(lane_base + col_s + 96, t1);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -267,97 +317,103 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int kv0 = j * kBN;
       const bool diag = CAUSAL && (j == n_kv - 1);
-      if (diag || kv0 + kBN > N) {
-        const int lim = min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN);  // visible keys
+      const bool masked = diag || kv0 + kBN > N;
+      const int lim = masked ? min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN) : kBN;
+      if (masked) {
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+      for (int c = 4; c < kBN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float m_cand = fmaxf(m, mx * scale_log2);
       const bool grow = m_cand > m + kRescaleLog2;  // true on the first tile
       const float alpha = grow ? ex2(m - m_cand) : 1.f;
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled.
-        const bool w2 = mbar_wait(o_done, (j - 1) & 1, abort, ctl, kSiteFwdSoftmax);
-        if (!__all_sync(0xffffffffu, w2)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        // O_x += P_x(j-1) V completed before S_x(j) (same MMA thread, in
+        // order), so O_x can be rescaled now.
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
           uint32_t o16[16];
-          tmem_ld16(lane_base + kColO + c * 16, o16);
+          tmem_ld16(lane_base + col_o + c * 16, o16);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
-          tmem_st16(lane_base + kColO + c * 16, o16);
+          tmem_st16(lane_base + col_o + c * 16, o16);
         }
-        tmem_wait_st();
       }
       if (grow) {
         l *= alpha;
         m = m_cand;
       }
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      float rs = 0.f;
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      // One column pair in three goes to the FMA-pipe exp2, the rest to the
+      // special-function unit, so the two units share the exponentials.
+      float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
       uint32_t pk[kBN / 2];
 #pragma unroll
       for (int c = 0; c < kBN / 2; ++c) {
-        const float p0 = ex2(fmaf(s[2 * c], scale_log2, neg_m));
-        const float p1 = ex2(fmaf(s[2 * c + 1], scale_log2, neg_m));
-        rs += p0 + p1;
-        pk[c] = pack_bf16(p0, p1);
+        const float2 xx = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+        float2 p;
+        if (c % 3 == 2) {
+          p = exp2_fma2(xx);
+          if (masked) {
+            if (2 * c >= lim) p.x = 0.f;
+            if (2 * c + 1 >= lim) p.y = 0.f;
+          }
+        } else {
+          p = make_float2(ex2(xx.x), ex2(xx.y));
+        }
+        rs2[c & 3] = __fadd2_rn(rs2[c & 3], p);
+        pk[c] = pack_bf16(p.x, p.y);
       }
+      const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+      const float rs = rsa.x + rsa.y;
       l += rs;
       {
         uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
         uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-        tmem_st32(lane_base + sb * kBN + 0, lo);
-        tmem_st32(lane_base + sb * kBN + 32, hi);
+        tmem_st32(lane_base + col_s + 0, lo);
+        tmem_st32(lane_base + col_s + 32, hi);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full + sb);
+      mbar_arrive(p_full + x);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) {
-      const bool w = mbar_wait(o_done, (n_kv - 1) & 1, abort, ctl, kSiteFwdEpilogue);
-      if (__all_sync(0xffffffffu, w)) {
-        tc_fence_after();
-        const float inv_l = 1.f / l;
-        const bool valid = q_idx < N;
-        uint4* orow = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
+    if (ok && n_kv > 0 && wait_all(o_done + x, (n_kv - 1) & 1, abort, ctl, kSiteFwdEpilogue)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool valid = q_idx < N;
+      uint4* orow = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t o16[16];
-          tmem_ld16(lane_base + kColO + c * 16, o16);
-          tmem_wait_ld();
-          uint4 a, b;
-          a.x = pack_bf16(__uint_as_float(o16[0]) * inv_l, __uint_as_float(o16[1]) * inv_l);
-          a.y = pack_bf16(__uint_as_float(o16[2]) * inv_l, __uint_as_float(o16[3]) * inv_l);
-          a.z = pack_bf16(__uint_as_float(o16[4]) * inv_l, __uint_as_float(o16[5]) * inv_l);
-          a.w = pack_bf16(__uint_as_float(o16[6]) * inv_l, __uint_as_float(o16[7]) * inv_l);
-          b.x = pack_bf16(__uint_as_float(o16[8]) * inv_l, __uint_as_float(o16[9]) * inv_l);
-          b.y = pack_bf16(__uint_as_float(o16[10]) * inv_l, __uint_as_float(o16[11]) * inv_l);
-          b.z = pack_bf16(__uint_as_float(o16[12]) * inv_l, __uint_as_float(o16[13]) * inv_l);
-          b.w = pack_bf16(__uint_as_float(o16[14]) * inv_l, __uint_as_float(o16[15]) * inv_l);
-          if (valid) {
-            orow[2 * c] = a;
-            orow[2 * c + 1] = b;
-          }
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t o16[16];
+        tmem_ld16(lane_base + col_o + c * 16, o16);
+        tmem_wait_ld();
+        uint32_t pkd[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          pkd[e] = pack_bf16(__uint_as_float(o16[2 * e]) * inv_l,
+                             __uint_as_float(o16[2 * e + 1]) * inv_l);
+        if (valid) {
+          orow[2 * c] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+          orow[2 * c + 1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
         }
-        if (valid) lse[static_cast<size_t>(bh) * N + q_idx] = (m + __log2f(l)) * 0.69314718055994531f;
       }
+      if (valid)
+        lse[static_cast<size_t>(bh) * N + q_idx] = (m + __log2f(l)) * 0.69314718055994531f;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -369,18 +425,25 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   using C = Cfg<D>;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, CAUSAL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    // The register split above assumes the kernel was compiled to exactly
+    // kLaunchRegs per thread; with fewer, the increase would wait forever.
+    cudaFuncAttributes fattr;
+    cudaError_t e = cudaFuncGetAttributes(&fattr, fwd_kernel<D, CAUSAL>);
+    if (e != cudaSuccess) return e;
+    if (fattr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(fwd_kernel<D, CAUSAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int n_qt = (N + kBM - 1) / kBM;
+  const int n_t = (N + kBM - 1) / kBM;
+  const int n_pair = (n_t + 1) / 2;
   // Heads per group: keep a group's Q, K, V and O (8 N d bytes per head)
   // within ~48 MB of the 126 MB L2.
   const long long per_head = 8LL * N * D;
   int group = static_cast<int>((48LL << 20) / (per_head > 0 ? per_head : 1));
   group = group < 1 ? 1 : (group > BH ? BH : group);
-  const long long blocks = static_cast<long long>(BH) * n_qt;
+  const long long blocks = static_cast<long long>(BH) * n_pair;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};

@@ -43,20 +43,20 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
                              void* o, float* lse, int BH, int N, int d, float scale, int causal,
                              const Launch& L);
 
-// tdq: the fp32 dQ accumulator [BH, N, d] as 3-D {d, N, BH}, box {32, 32, 1},
-// 128-byte swizzle (target of the TMA reductions).
+// Backward: the dK/dV kernel then the dQ kernel, both in stream order.
+// dvec and lse2 are the preprocess outputs ([BH, Np] fp32, Np = N rounded up
+// to 128); dq, dk, dv are bf16 [BH, N, d] outputs.
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tdo, const CUtensorMap& tdq, const float* dvec,
-                             const float* lse2, void* dk, void* dv, int BH, int N, int d,
-                             float scale, int causal, const Launch& L);
+                             const CUtensorMap& tdo, const float* dvec, const float* lse2,
+                             void* dq, void* dk, void* dv, int BH, int N, int d, float scale,
+                             int causal, const Launch& L);
 
 // --- helpers shared by both dtypes (fa_simt.cu) ---------------------------
-// D = rowsum(dO o O) (fp32, padded rows = 0), lse2 = LSE * log2(e) (padded
-// rows = +inf), and zero the fp32 dQ accumulator.
+// D = rowsum(dO o O) (fp32, padded rows = 0) and, when lse2 is non-null,
+// lse2 = LSE * log2(e) (padded rows = +inf).
 cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse, float* dvec,
-                                  float* lse2, float* dq_acc, int BH, int N, int d, int is_bf16,
+                                  float* lse2, int BH, int N, int d, int is_bf16,
                                   const Launch& L);
-cudaError_t launch_dq_convert_bf16(const float* dq_acc, void* dq, size_t n, const Launch& L);
 
 // --- fp32 SIMT path (fa_simt.cu) -------------------------------------------
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,

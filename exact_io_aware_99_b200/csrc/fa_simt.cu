@@ -2,8 +2,7 @@
 //   * the fp32 forward and backward (fp32 FMA throughout, for accuracy
 //     checks at small sizes; TF32 tensor cores cannot hold 1e-5),
 //   * the backward preprocess shared by both dtypes
-//     (D = rowsum(dO o O), base-2 LSE, zeroing the fp32 dQ accumulator),
-//   * the fp32 -> bf16 dQ conversion,
+//     (D = rowsum(dO o O) and the base-2 LSE, padded to whole 128-row tiles),
 //   * the bounded-wait self test.
 //
 // The forward follows the blocked algorithm of the "FlashAttention-2" review
@@ -240,8 +239,7 @@ __device__ __forceinline__ float ld_as_float<__nv_bfloat16>(const __nv_bfloat16*
 template <typename T>
 __global__ void bwd_preprocess_kernel(const T* __restrict__ o, const T* __restrict__ dO,
                                       const float* __restrict__ lse, float* __restrict__ dvec,
-                                      float* __restrict__ lse2, float* __restrict__ dq_acc, int BH,
-                                      int N, int Np, int d) {
+                                      float* __restrict__ lse2, int BH, int N, int Np, int d) {
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= BH * Np) return;
@@ -252,7 +250,6 @@ __global__ void bwd_preprocess_kernel(const T* __restrict__ o, const T* __restri
     const size_t base = (static_cast<size_t>(bh) * N + row) * d;
     for (int c = lane; c < d; c += 32) {
       acc = fmaf(ld_as_float(dO, base + c), ld_as_float(o, base + c), acc);
-      if (dq_acc) dq_acc[base + c] = 0.f;
     }
   }
 #pragma unroll
@@ -262,18 +259,6 @@ __global__ void bwd_preprocess_kernel(const T* __restrict__ o, const T* __restri
     dvec[vi] = row < N ? acc : 0.f;
     if (lse2)
       lse2[vi] = row < N ? lse[static_cast<size_t>(bh) * N + row] * 1.4426950408889634f : INFINITY;
-  }
-}
-
-__global__ void dq_convert_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
-                                  size_t n4) {
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const float4 a = src[i];
-    uint2 r;
-    r.x = pack_bf16(a.x, a.y);
-    r.y = pack_bf16(a.z, a.w);
-    dst[i] = r;
   }
 }
 
@@ -335,7 +320,7 @@ cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const
 }
 
 cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse, float* dvec,
-                                  float* lse2, float* dq_acc, int BH, int N, int d, int is_bf16,
+                                  float* lse2, int BH, int N, int d, int is_bf16,
                                   const Launch& L) {
   const int Np = round_up(N, kTileRows);
   const size_t warps = static_cast<size_t>(BH) * Np;
@@ -344,21 +329,11 @@ cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* ls
   if (is_bf16)
     simt::bwd_preprocess_kernel<__nv_bfloat16><<<blocks, threads, 0, L.stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
-        lse2, dq_acc, BH, N, Np, d);
+        lse2, BH, N, Np, d);
   else
     simt::bwd_preprocess_kernel<float><<<blocks, threads, 0, L.stream>>>(
-        static_cast<const float*>(o), static_cast<const float*>(dO), lse, dvec, lse2, dq_acc, BH,
-        N, Np, d);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dq_convert_bf16(const float* dq_acc, void* dq, size_t n, const Launch& L) {
-  const size_t n4 = n / 4;  // n is a multiple of 16 (d in {64, 80, 128})
-  const int threads = 256;
-  int blocks = blocks_for(n4, threads);
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  simt::dq_convert_kernel<<<blocks, threads, 0, L.stream>>>(
-      reinterpret_cast<const float4*>(dq_acc), static_cast<uint2*>(dq), n4);
+        static_cast<const float*>(o), static_cast<const float*>(dO), lse, dvec, lse2, BH, N, Np,
+        d);
   return cudaGetLastError();
 }
 

@@ -99,6 +99,17 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* m, uint64_t* bar,
       : "memory");
 }
 
+// Contiguous (untiled) bulk copy global -> shared, completion as transaction
+// bytes on `bar`.  Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 3-D tiled reduction (element-wise add, no multicast) of a shared-memory box
 // into global memory; completion is tracked with bulk groups.
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* src, int x,
@@ -119,6 +130,11 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 // Wait until all committed bulk groups have completed.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Hint: bring the 128-byte line holding `p` into L1 (no register, no wait).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
 // Make generic-proxy writes to shared memory visible to the async proxy
@@ -264,6 +280,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// Warpgroup register re-allocation.  The block's register budget is fixed at
+// launch (threads x registers per thread); every warpgroup of the block must
+// execute one of these, and the shares must add up to at most that budget.
+template <int R>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 // ------------------------------------------------------------ arithmetic
 
 // 2^x on the special-function unit (approximate, flush-to-zero).
@@ -271,6 +299,31 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for two values on the FMA pipe (no special-function unit):
+// 2^x = 2^n 2^f with n = round(x) (via the 1.5 * 2^23 shifter) and
+// f = x - n in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients
+// are the relative-error minimax fit on [-1/2, 1/2] computed by
+// exact_io_aware_99_b200/fit_exp2.py (max relative error 7.5e-5); 2^n is
+// added to the exponent field.  x is clamped to -126, so very negative
+// arguments (and -inf) give about 1.2e-38 rather than 0: callers zero masked
+// entries themselves.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+  constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+  p.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
+  p.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
+  return p;
 }
 
 // Pack two floats to bf16x2 (round to nearest even): `lo` in bits 0..15.

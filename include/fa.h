@@ -105,10 +105,11 @@ FA_API fa_status fa_forward_ex(const void* q, const void* k, const void* v, void
 
 /*
  * fa_backward_workspace_size -- bytes of device scratch fa_backward needs:
- * an fp32 dQ accumulator [B, H, N, d] plus two fp32 row vectors per head
- * padded to a multiple of 128 rows (D = rowsum(dO o O) and the base-2 LSE),
- * each part rounded up to 256 bytes.  Linear in N (no N x N buffer).
- * Returns 0 for arguments that fa_backward would reject.
+ * two fp32 row vectors per head padded to a multiple of 128 rows
+ * (D = rowsum(dO o O) and the base-2 LSE), each rounded up to 256 bytes:
+ * 2 * round256(4 * B * H * ceil(N / 128) * 128).  Linear in N (no N x N
+ * buffer); independent of d.  Returns 0 for arguments that fa_backward would
+ * reject.
  */
 FA_API size_t fa_backward_workspace_size(int B, int H, int N, int d);
 
@@ -123,7 +124,10 @@ FA_API size_t fa_backward_workspace_size(int B, int H, int N, int d);
  *                   not matter and are clobbered.  Two calls that overlap on
  *                   the GPU must not share one workspace.
  *   Other arguments as in fa_forward (same scale and causal as the forward).
- * Launches three kernels in stream order (preprocess, main, dQ convert).
+ * Launches three kernels in stream order: the preprocess (D and the base-2
+ * LSE), the dK/dV kernel and the dQ kernel.  dQ is computed by its own kernel
+ * (it recomputes S and dP per query tile), so no atomics are used and the
+ * result is bitwise reproducible.
  */
 FA_API fa_status fa_backward(const void* q, const void* k, const void* v,
                       const void* o, const void* dO, const float* lse,

@@ -54,7 +54,7 @@ def test_noalloc_backward_rejects_problems_larger_than_its_scratch():
     # Rejected on the host before any device work (fake, aligned pointers).
     import exact_io_aware_99_b200 as fa
     A = 1 << 20
-    B, H, N, d = 1, 16, 16384, 128
+    B, H, N, d = 64, 64, 4096, 128
     assert fa.fa_backward_workspace_size(B, H, N, d) > fa.FA_NOALLOC_SCRATCH_BYTES
     st = fa.fa_backward_noalloc(A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 7 * A, 8 * A, 9 * A,
                                 B, H, N, d, 0.1, 1, stream=0, check=False)
