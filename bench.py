@@ -5,14 +5,14 @@
                     [--impl ours|reference] [--no-cpu-baseline] [--sweep]
 
 One step is one pass of the whole hot path over one batch: the forward
-(fa_forward: O and LSE) followed by the backward (fa_backward: D
-preprocess, the dK/dV/dQ kernel, the dQ conversion) of the workload, inputs
+(fa_forward: O and LSE) followed by the backward (fa_backward: the D / LSE2
+preprocess, the dK/dV kernel and the dQ kernel) of the workload, inputs
 resident in HBM.  Throughput counts the algorithmic FLOPs of both passes
 (forward 4 B H N^2 d, halved when causal; backward 2.5x the forward).
 
 Default workload: causal_d128 (B4 H16 N4096 d128, bf16, causal fwd+bwd),
 the configuration the metric's target is stated at (N >= 4096, d = 128).
-Its working set (~0.7 GB) is larger than the 126 MB L2, so no flush is needed
+Its working set (~0.5 GB) is larger than the 126 MB L2, so no flush is needed
 between steps.  Under torchrun each rank runs the same per-GPU workload on its
 own GPU (independent heads, no collective on the data path: weak scaling);
 the time is the max over ranks.
@@ -127,7 +127,8 @@ class ClockSampler:
 # --------------------------------------------------------------- ncu traffic
 
 KERNEL_SOURCES = {
-    "bwd": ["exact_io_aware_99_b200/csrc/fa_bwd_sm100.cu", "exact_io_aware_99_b200/csrc/sm100.cuh"],
+    "bwd": ["exact_io_aware_99_b200/csrc/fa_bwd_sm100.cu", "exact_io_aware_99_b200/csrc/fa_simt.cu",
+            "exact_io_aware_99_b200/csrc/sm100.cuh"],
     "fwd": ["exact_io_aware_99_b200/csrc/fa_fwd_sm100.cu", "exact_io_aware_99_b200/csrc/sm100.cuh"],
 }
 
