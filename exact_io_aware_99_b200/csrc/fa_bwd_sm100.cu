@@ -250,19 +250,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S^T, dP^T
       constexpr uint32_t kIdescAcc = idesc_bf16(kT, D, 0, 1);  // dV, dK (B MN-major)
-      const uint32_t k_addr = sbase + C::K_OFF;
-      const uint32_t v_addr = sbase + C::V_OFF;
+      const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);           // K-major (A)
+      const SDesc v_desc = sdesc(sbase + C::V_OFF, 16, 1024);           // K-major (A)
+      const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);           // K-major (B of S^T)
+      const SDesc do_desc = sdesc(sbase + C::DO_OFF, 16, 1024);         // K-major (B of dP^T)
+      const SDesc q_mn = sdesc(sbase + C::Q_OFF, C::BLK, 1024);         // MN-major (B of dK)
+      const SDesc do_mn = sdesc(sbase + C::DO_OFF, C::BLK, 1024);       // MN-major (B of dV)
       auto issue_s = [&](int it) -> bool {  // S^T = K_j Q_i^T -> region A
         const int st = it & 1;
         if (!mbar_wait(q_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
           return false;
         tc_fence_after();
-        const uint32_t q_addr = sbase + C::Q_OFF + st * C::TILE;
+        const SDesc qd = q_desc + st * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kKvColS, sdesc_sw128(k_addr + off, 16, 1024),
-                 sdesc_sw128(q_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kKvColS, k_desc + off, qd + off, kIdescSq, kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full);
         return true;
@@ -272,12 +275,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(do_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
           return false;
         tc_fence_after();
-        const uint32_t do_addr = sbase + C::DO_OFF + st * C::TILE;
+        const SDesc dd = do_desc + st * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kKvColDP, sdesc_sw128(v_addr + off, 16, 1024),
-                 sdesc_sw128(do_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kKvColDP, v_desc + off, dd + off, kIdescSq, kk > 0 ? 1u : 0u);
         }
         mma_commit(dp_full);
         return true;
@@ -288,8 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(kv_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
       for (int it = 0; ok && it < n_iter; ++it) {
         const int st = it & 1;
-        const uint32_t q_addr = sbase + C::Q_OFF + st * C::TILE;
-        const uint32_t do_addr = sbase + C::DO_OFF + st * C::TILE;
+        const SDesc qm = q_mn + st * C::TILE;
+        const SDesc dm = do_mn + st * C::TILE;
         // dV += P^T dO_i: query k-step kk (16 queries) lives in columns
         // 64*(kk/4) + 8*(kk%4) of region A.
         if (!mbar_wait(p_full, it & 1, abort, ctl, kSiteBwdMma)) break;
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
           mma_ts(tmem + kKvColDV, tmem + kKvColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                 sdesc_sw128(do_addr + kk * 2048, C::BLK, 1024), kIdescAcc,
+                 dm + kk * 2048, kIdescAcc,
                  (it > 0 || kk > 0) ? 1u : 0u);
         if (!mbar_wait(ds_full, it & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
           mma_ts(tmem + kKvColDK, tmem + kKvColDP + (kk >> 2) * 64 + (kk & 3) * 8,
-                 sdesc_sw128(q_addr + kk * 2048, C::BLK, 1024), kIdescAcc,
+                 qm + kk * 2048, kIdescAcc,
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(qdo_empty + st);
         if (it + 1 < n_iter && !issue_dp(it + 1)) break;
@@ -573,18 +575,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S, dP
       constexpr uint32_t kIdescDq = idesc_bf16(kT, D, 0, 1);   // dQ (B = K_j MN-major)
-      const uint32_t q_addr = sbase + C::Q_OFF;
-      const uint32_t do_addr = sbase + C::DO_OFF;
+      const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);     // K-major (A of S)
+      const SDesc do_desc = sdesc(sbase + C::DO_OFF, 16, 1024);   // K-major (A of dP)
+      const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);     // K-major (B of S)
+      const SDesc v_desc = sdesc(sbase + C::V_OFF, 16, 1024);     // K-major (B of dP)
+      const SDesc k_mn = sdesc(sbase + C::K_OFF, C::BLK, 1024);   // MN-major (B of dQ)
       auto issue_s = [&](int jj) -> bool {  // S_jj = Q K_jj^T -> buffer jj % 2
         const int s = jj % C::NK;
         if (!mbar_wait(k_full + s, (jj / C::NK) & 1, abort, ctl, kSiteBwdMma)) return false;
         tc_fence_after();
-        const uint32_t k_addr = sbase + C::K_OFF + s * C::TILE;
+        const SDesc kd = k_desc + s * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kQColS + (jj & 1) * kT, sdesc_sw128(q_addr + off, 16, 1024),
-                 sdesc_sw128(k_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kQColS + (jj & 1) * kT, q_desc + off, kd + off, kIdescSq,
+                 kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full + (jj & 1));
         return true;
@@ -593,12 +598,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = jj % C::NV;
         if (!mbar_wait(v_full + s, (jj / C::NV) & 1, abort, ctl, kSiteBwdMma)) return false;
         tc_fence_after();
-        const uint32_t v_addr = sbase + C::V_OFF + s * C::TILE;
+        const SDesc vd = v_desc + s * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kQColDP, sdesc_sw128(do_addr + off, 16, 1024),
-                 sdesc_sw128(v_addr + off, 16, 1024), kIdescSq, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kQColDP, do_desc + off, vd + off, kIdescSq, kk > 0 ? 1u : 0u);
         }
         mma_commit(dp_full);
         mma_commit(v_empty + s);
@@ -614,13 +618,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = jj % C::NK;
         if (!mbar_wait(ds_full + (jj & 1), (jj >> 1) & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
-        const uint32_t k_addr = sbase + C::K_OFF + s * C::TILE;
+        const SDesc km = k_mn + s * C::TILE;
         // dQ += dS_jj K_jj: key k-step kk (16 keys) of dS at column
         // 64*(kk/4) + 8*(kk%4) of the S buffer.
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
           mma_ts(tmem + kQColDQ, tmem + kQColS + (jj & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
-                 sdesc_sw128(k_addr + kk * 2048, C::BLK, 1024), kIdescDq,
+                 km + kk * 2048, kIdescDq,
                  (jj > 0 || kk > 0) ? 1u : 0u);
         mma_commit(k_empty + s);
         if (jj + 1 < n_kv && !issue_dp(jj + 1)) break;

@@ -50,6 +50,9 @@ constexpr int kThreads = 384;         // 2 softmax warpgroups + producer/MMA war
 constexpr int kLaunchRegs = 168, kSoftmaxRegs = 224, kControlRegs = 56;
 static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kLaunchRegs, "register split over budget");
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
+#ifndef FA_FWD_POLY_EVERY
+#define FA_FWD_POLY_EVERY 0  // one column pair in this many uses the FMA-pipe exp2 (0: none)
+#endif
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -62,7 +65,7 @@ struct Cfg {
   static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + NST * TILE;
   static constexpr int BAR_OFF = V_OFF + NST * TILE;
-  static constexpr int NBAR = 1 + 4 * NST + 6;
+  static constexpr int NBAR = 1 + 4 * NST + 6 + 8;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;  // + slack for 1 KB alignment
   static constexpr int KSTEPS = D / 16;
@@ -109,6 +112,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = v_empty + C::NST;  // [2] per tile
   uint64_t* p_full = s_full + 2;        // [2] per tile
   uint64_t* o_done = p_full + 2;        // [2] per tile
+  // Exponential-phase tokens between the two warps that share an SM
+  // sub-partition (warp w of tile A, warp w + 4 of tile B): tok_ab[w] says
+  // "A's warp w finished exp(j)", tok_ba[w] "B's warp w finished exp(j)".
+  uint64_t* tok_ab = o_done + 2;        // [4]
+  uint64_t* tok_ba = tok_ab + 4;        // [4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -148,6 +156,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(s_full + x, 1);
       mbar_init(p_full + x, kBM);
       mbar_init(o_done + x, 1);
+    }
+    for (int w = 0; w < 4; ++w) {
+      mbar_init(tok_ab + w, 1);
+      mbar_init(tok_ba + w, 1);
     }
     *abort = 0;
     fence_barrier_init();
@@ -223,23 +235,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         return true;
       };
+      const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);       // K-major
+      const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);       // K-major
+      const SDesc v_desc = sdesc(sbase + C::V_OFF, C::BLK, 1024);   // MN-major
       auto issue_s = [&](int x, int jj) {  // S_x = Q_x K_jj^T
-        const uint32_t q_addr = sbase + C::Q_OFF + x * C::TILE;
-        const uint32_t k_addr = sbase + C::K_OFF + (jj % C::NST) * C::TILE;
+        const SDesc qd = q_desc + x * C::TILE;
+        const SDesc kd = k_desc + (jj % C::NST) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + x * kBN, sdesc_sw128(q_addr + off, 16, 1024),
-                 sdesc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + x * kBN, qd + off, kd + off, kIdescS, kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full + x);
       };
       auto issue_pv = [&](int x, int jj) {  // O_x += P_x V_jj, P_x from TMEM
-        const uint32_t v_addr = sbase + C::V_OFF + (jj % C::NST) * C::TILE;
+        const SDesc vd = v_desc + (jj % C::NST) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_ts(tmem + 256 + x * kBN, tmem + x * kBN + kk * 8,
-                 sdesc_sw128(v_addr + kk * 16 * 128, C::BLK, 1024), kIdescPV,
+                 vd + kk * 16 * 128, kIdescPV,
                  (jj > 0 || kk > 0) ? 1u : 0u);
         mma_commit(o_done + x);
       };
@@ -348,11 +362,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         m = m_cand;
       }
+      // The two tiles' warps on one sub-partition take turns on the MUFU:
+      // A(0), B(0), A(1), B(1), ...  (only while both tiles still run).
+      const int wq = warp & 3;
+      if (x == 0 ? (j >= 1 && j - 1 < n_x[1]) : (j < n_x[0])) {
+        uint64_t* tok = x == 0 ? tok_ba + wq : tok_ab + wq;
+        const uint32_t par = static_cast<uint32_t>(x == 0 ? j - 1 : j) & 1;
+        if (!wait_all(tok, par, abort, ctl, kSiteFwdSoftmax)) {
+          ok = false;
+          break;
+        }
+      }
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       const float2 sc2 = make_float2(scale_log2, scale_log2);
       const float2 nm2 = make_float2(neg_m, neg_m);
-      // One column pair in three goes to the FMA-pipe exp2, the rest to the
-      // special-function unit, so the two units share the exponentials.
+      // One column pair in FA_FWD_POLY_EVERY goes to the FMA-pipe exp2, the
+      // rest to the special-function unit, so the two units share the work.
       float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
       uint32_t pk[kBN / 2];
@@ -360,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < kBN / 2; ++c) {
         const float2 xx = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
         float2 p;
-        if (c % 3 == 2) {
+        if (FA_FWD_POLY_EVERY > 0 && c % FA_FWD_POLY_EVERY == FA_FWD_POLY_EVERY - 1) {
           p = exp2_fma2(xx);
           if (masked) {
             if (2 * c >= lim) p.x = 0.f;
@@ -374,6 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
       const float rs = rsa.x + rsa.y;
+      __syncwarp();
+      if (lane == 0 && (x == 0 ? (j < n_x[1]) : (j + 1 < n_x[0])))
+        mbar_arrive(x == 0 ? tok_ab + wq : tok_ba + wq);
       l += rs;
       {
         uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);

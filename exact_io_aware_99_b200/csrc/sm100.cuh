@@ -51,12 +51,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
+  // The suspend-time hint lets a waiting warp sleep in the barrier unit
+  // instead of re-issuing the test, leaving issue slots to the warps of its
+  // sub-partition that have work (the MMA issuer, the softmax).
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.b32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(20000u)
       : "memory");
   return ok != 0;
 }
@@ -172,25 +175,53 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Shared-memory matrix descriptor as two 32-bit words.  The issuing thread
+// builds each operand family's descriptor once and advances it per k-step
+// or stage by adding the byte offset / 16 to the low word (the 14-bit start
+// address field; shared addresses stay below 256 KB, so no carry leaves it).
+// Keeping the per-MMA work to an add is what lets a single thread that shares
+// its sub-partition with busy softmax warps keep the tensor core fed.
+struct SDesc {
+  uint32_t lo, hi;
+};
+// 128-byte-swizzled operand at shared address `saddr`.
+//   K-major tile: rows of 64 bf16 (128 B), 8-row groups 1024 B apart (SBO);
+//                 LBO unused (16).  A k-step of 16 elements advances 32 B.
+//   MN-major tile: 64 MN-contiguous elements per 128-B row, one row per k;
+//                 8-k groups SBO apart, 64-wide MN atoms LBO apart.
+__device__ __forceinline__ SDesc sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  SDesc d;
+  d.lo = ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+  d.hi = ((sbo >> 4) & 0x3FFFu) | (1u << 14) /* version (sm_100) */ | (2u << 29) /* 128B swizzle */;
+  return d;
+}
+__device__ __forceinline__ SDesc operator+(SDesc d, uint32_t bytes) {
+  d.lo += bytes >> 4;
+  return d;
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, one 16-deep k-step, bf16 in, fp32 acc.
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, SDesc a, SDesc b, uint32_t idesc,
+                                       uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
 // D[tmem] (+)= A[tmem] * B[smem], A read from tensor memory (K-major).
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, SDesc b, uint32_t idesc,
+                                       uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -213,22 +244,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          | (static_cast<uint32_t>(b_mn) << 16)  // B major
          | (static_cast<uint32_t>(N >> 3) << 17)
          | (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-// Shared-memory matrix descriptor for a 128-byte-swizzled operand.
-//   K-major tile: rows of 64 bf16 (128 B), 8-row groups 1024 B apart (SBO);
-//                 LBO unused (1).  A k-step of 16 elements advances the
-//                 start address by 32 B inside the swizzle atom.
-//   MN-major tile: 64 MN-contiguous elements per 128-B row, one row per k;
-//                 8-k groups SBO apart, 64-wide MN atoms LBO apart.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
-  d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm_100)
-  d |= static_cast<uint64_t>(2) << 61;  // 128-byte swizzle
-  return d;
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets
