@@ -37,8 +37,8 @@
 // Warp roles (both kernels, 10 warps): warps 0-3 and 4-7 are two softmax
 // warpgroups splitting the 128 columns of every tile in halves (one thread
 // per TMEM lane), warp 8 is the TMA producer, warp 9 the TMEM allocator and
-// single-thread MMA issuer.  CTAs run group-major (a few heads at a time, so
-// their operands stay in L2), longest-first inside a group.
+// MMA issuer (one elected lane).  CTAs run group-major (a few heads at a
+// time, so their operands stay in L2), longest-first inside a group.
 #include <cuda_bf16.h>
 
 #include "fa_internal.h"
@@ -247,7 +247,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // All lanes run the schedule; the elected lane issues MMAs and commits.
+    {
+      const bool leader = elect_one();
       constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S^T, dP^T
       constexpr uint32_t kIdescAcc = idesc_bf16(kT, D, 0, 1);  // dV, dK (B MN-major)
       const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);           // K-major (A)
@@ -258,62 +260,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       const SDesc do_mn = sdesc(sbase + C::DO_OFF, C::BLK, 1024);       // MN-major (B of dV)
       auto issue_s = [&](int it) -> bool {  // S^T = K_j Q_i^T -> region A
         const int st = it & 1;
-        if (!mbar_wait(q_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
+        if (!wait_all(q_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
           return false;
         tc_fence_after();
-        const SDesc qd = q_desc + st * C::TILE;
+        if (leader) {
+          const SDesc qd = q_desc + st * C::TILE;
 #pragma unroll
-        for (int kk = 0; kk < C::KSTEPS; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kKvColS, k_desc + off, qd + off, kIdescSq, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+            mma_ss(tmem + kKvColS, k_desc + off, qd + off, kIdescSq, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full);
         }
-        mma_commit(s_full);
+        __syncwarp();
         return true;
       };
       auto issue_dp = [&](int it) -> bool {  // dP^T = V_j dO_i^T -> region B
         const int st = it & 1;
-        if (!mbar_wait(do_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
+        if (!wait_all(do_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
           return false;
         tc_fence_after();
-        const SDesc dd = do_desc + st * C::TILE;
+        if (leader) {
+          const SDesc dd = do_desc + st * C::TILE;
 #pragma unroll
-        for (int kk = 0; kk < C::KSTEPS; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kKvColDP, v_desc + off, dd + off, kIdescSq, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+            mma_ss(tmem + kKvColDP, v_desc + off, dd + off, kIdescSq, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(dp_full);
         }
-        mma_commit(dp_full);
+        __syncwarp();
         return true;
       };
       // S^T_{i+1} overwrites P^T_i in A: issued after dV_i (same thread, in
       // order) and after the softmax finished reading P^T_i (ds_full).
       // dP^T_{i+1} overwrites dS^T_i in B: issued after dK_i, in order.
-      bool ok = mbar_wait(kv_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
+      bool ok = wait_all(kv_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
       for (int it = 0; ok && it < n_iter; ++it) {
         const int st = it & 1;
         const SDesc qm = q_mn + st * C::TILE;
         const SDesc dm = do_mn + st * C::TILE;
         // dV += P^T dO_i: query k-step kk (16 queries) lives in columns
         // 64*(kk/4) + 8*(kk%4) of region A.
-        if (!mbar_wait(p_full, it & 1, abort, ctl, kSiteBwdMma)) break;
+        if (!wait_all(p_full, it & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk)
-          mma_ts(tmem + kKvColDV, tmem + kKvColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                 dm + kk * 2048, kIdescAcc,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        if (!mbar_wait(ds_full, it & 1, abort, ctl, kSiteBwdMma)) break;
+          for (int kk = 0; kk < kT / 16; ++kk)
+            mma_ts(tmem + kKvColDV, tmem + kKvColS + (kk >> 2) * 64 + (kk & 3) * 8,
+                   dm + kk * 2048, kIdescAcc,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
+        if (!wait_all(ds_full, it & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
         if (it + 1 < n_iter && !issue_s(it + 1)) break;
         // dK += dS^T Q_i: dS^T k-step kk at column 128 + 64*(kk/4) + 8*(kk%4).
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk)
-          mma_ts(tmem + kKvColDK, tmem + kKvColDP + (kk >> 2) * 64 + (kk & 3) * 8,
-                 qm + kk * 2048, kIdescAcc,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(qdo_empty + st);
+          for (int kk = 0; kk < kT / 16; ++kk)
+            mma_ts(tmem + kKvColDK, tmem + kKvColDP + (kk >> 2) * 64 + (kk & 3) * 8,
+                   qm + kk * 2048, kIdescAcc,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(qdo_empty + st);
+        }
+        __syncwarp();
         if (it + 1 < n_iter && !issue_dp(it + 1)) break;
       }
-      mma_commit(kv_done);
+      if (leader) mma_commit(kv_done);
     }
     __syncwarp();
   } else {
@@ -572,7 +586,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // All lanes run the schedule; the elected lane issues MMAs and commits.
+    {
+      const bool leader = elect_one();
       constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S, dP
       constexpr uint32_t kIdescDq = idesc_bf16(kT, D, 0, 1);   // dQ (B = K_j MN-major)
       const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);     // K-major (A of S)
@@ -582,55 +598,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       const SDesc k_mn = sdesc(sbase + C::K_OFF, C::BLK, 1024);   // MN-major (B of dQ)
       auto issue_s = [&](int jj) -> bool {  // S_jj = Q K_jj^T -> buffer jj % 2
         const int s = jj % C::NK;
-        if (!mbar_wait(k_full + s, (jj / C::NK) & 1, abort, ctl, kSiteBwdMma)) return false;
+        if (!wait_all(k_full + s, (jj / C::NK) & 1, abort, ctl, kSiteBwdMma)) return false;
         tc_fence_after();
-        const SDesc kd = k_desc + s * C::TILE;
+        if (leader) {
+          const SDesc kd = k_desc + s * C::TILE;
 #pragma unroll
-        for (int kk = 0; kk < C::KSTEPS; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kQColS + (jj & 1) * kT, q_desc + off, kd + off, kIdescSq,
-                 kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+            mma_ss(tmem + kQColS + (jj & 1) * kT, q_desc + off, kd + off, kIdescSq,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full + (jj & 1));
         }
-        mma_commit(s_full + (jj & 1));
+        __syncwarp();
         return true;
       };
       auto issue_dp = [&](int jj) -> bool {  // dP_jj = dO V_jj^T, then V_jj is free
         const int s = jj % C::NV;
-        if (!mbar_wait(v_full + s, (jj / C::NV) & 1, abort, ctl, kSiteBwdMma)) return false;
+        if (!wait_all(v_full + s, (jj / C::NV) & 1, abort, ctl, kSiteBwdMma)) return false;
         tc_fence_after();
-        const SDesc vd = v_desc + s * C::TILE;
+        if (leader) {
+          const SDesc vd = v_desc + s * C::TILE;
 #pragma unroll
-        for (int kk = 0; kk < C::KSTEPS; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kQColDP, do_desc + off, vd + off, kIdescSq, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+            mma_ss(tmem + kQColDP, do_desc + off, vd + off, kIdescSq, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(dp_full);
+          mma_commit(v_empty + s);
         }
-        mma_commit(dp_full);
-        mma_commit(v_empty + s);
+        __syncwarp();
         return true;
       };
       // Order: S_0, dP_0, S_1, [dS_0] dQ_0, dP_1, S_2, [dS_1] dQ_1, ... so the
       // tensor core computes S_{j+1} while the softmax warps form dS_j.  S_{j+2}
       // reuses S_j's buffer after dQ_j has read dS_j (same thread, in order)
       // and the softmax released it (ds_full waited); dP_{j+1} likewise.
-      bool ok = mbar_wait(q_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
+      bool ok = wait_all(q_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
       if (ok && n_kv > 1) ok = issue_s(1);
       for (int jj = 0; ok && jj < n_kv; ++jj) {
         const int s = jj % C::NK;
-        if (!mbar_wait(ds_full + (jj & 1), (jj >> 1) & 1, abort, ctl, kSiteBwdMma)) break;
+        if (!wait_all(ds_full + (jj & 1), (jj >> 1) & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
-        const SDesc km = k_mn + s * C::TILE;
         // dQ += dS_jj K_jj: key k-step kk (16 keys) of dS at column
         // 64*(kk/4) + 8*(kk%4) of the S buffer.
+        if (leader) {
+          const SDesc km = k_mn + s * C::TILE;
 #pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk)
-          mma_ts(tmem + kQColDQ, tmem + kQColS + (jj & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
-                 km + kk * 2048, kIdescDq,
-                 (jj > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(k_empty + s);
+          for (int kk = 0; kk < kT / 16; ++kk)
+            mma_ts(tmem + kQColDQ, tmem + kQColS + (jj & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
+                   km + kk * 2048, kIdescDq,
+                   (jj > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(k_empty + s);
+        }
+        __syncwarp();
         if (jj + 1 < n_kv && !issue_dp(jj + 1)) break;
         if (jj + 2 < n_kv && !issue_s(jj + 2)) break;
       }
-      mma_commit(dq_done);
+      if (leader) mma_commit(dq_done);
     }
     __syncwarp();
   } else {

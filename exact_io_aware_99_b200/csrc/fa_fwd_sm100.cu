@@ -17,7 +17,7 @@
 //   warp 8      TMA producer: both Q tiles once, then K_j and V_j into
 //               separate shared-memory rings; each K/V tile serves both Q
 //               tiles (half the K/V traffic per FLOP of a one-tile CTA).
-//   warp 9      TMEM allocator and single-thread MMA issuer, alternating
+//   warp 9      TMEM allocator and MMA issuer (one elected lane), alternating
 //               between the tiles: O_A += P_A V_j, S_A = Q_A K_{j+1}^T,
 //               O_B += P_B V_j, S_B = Q_B K_{j+1}^T, so the tensor core works
 //               on one tile while the other tile's softmax runs.
@@ -223,22 +223,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, 0, 0);
-      constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, 0, 1);
-      int k_seen = -1;  // highest key tile whose k_full wait has been done
-      auto wait_k = [&](int jj) -> bool {
-        if (jj <= k_seen) return true;
-        if (!mbar_wait(k_full + jj % C::NST, (jj / C::NST) & 1, abort, ctl, kSiteFwdMma))
-          return false;
-        k_seen = jj;
-        tc_fence_after();
-        return true;
-      };
-      const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);       // K-major
-      const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);       // K-major
-      const SDesc v_desc = sdesc(sbase + C::V_OFF, C::BLK, 1024);   // MN-major
-      auto issue_s = [&](int x, int jj) {  // S_x = Q_x K_jj^T
+    // The whole warp runs the schedule (waits and branches stay uniform);
+    // the elected lane issues the MMAs and commits.
+    const bool leader = elect_one();
+    constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, 0, 0);
+    constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, 0, 1);
+    int k_seen = -1;  // highest key tile whose k_full wait has been done
+    auto wait_k = [&](int jj) -> bool {
+      if (jj <= k_seen) return true;
+      if (!wait_all(k_full + jj % C::NST, (jj / C::NST) & 1, abort, ctl, kSiteFwdMma))
+        return false;
+      k_seen = jj;
+      tc_fence_after();
+      return true;
+    };
+    const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);       // K-major
+    const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);       // K-major
+    const SDesc v_desc = sdesc(sbase + C::V_OFF, C::BLK, 1024);   // MN-major
+    auto issue_s = [&](int x, int jj) {  // S_x = Q_x K_jj^T
+      if (leader) {
         const SDesc qd = q_desc + x * C::TILE;
         const SDesc kd = k_desc + (jj % C::NST) * C::TILE;
 #pragma unroll
@@ -247,46 +250,53 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + x * kBN, qd + off, kd + off, kIdescS, kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full + x);
-      };
-      auto issue_pv = [&](int x, int jj) {  // O_x += P_x V_jj, P_x from TMEM
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int x, int jj) {  // O_x += P_x V_jj, P_x from TMEM
+      if (leader) {
         const SDesc vd = v_desc + (jj % C::NST) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + 256 + x * kBN, tmem + x * kBN + kk * 8,
-                 vd + kk * 16 * 128, kIdescPV,
+          mma_ts(tmem + 256 + x * kBN, tmem + x * kBN + kk * 8, vd + kk * 16 * 128, kIdescPV,
                  (jj > 0 || kk > 0) ? 1u : 0u);
         mma_commit(o_done + x);
-      };
-      bool ok = mbar_wait(q_full, 0, abort, ctl, kSiteFwdMma) && wait_k(0);
-      if (ok) {
-        tc_fence_after();
-        for (int x = 0; x < 2; ++x)
-          if (n_x[x] > 0) issue_s(x, 0);
-        mma_commit(k_empty + 0);
       }
-      for (int j = 0; ok && j < n_max; ++j) {
-        const int s = j % C::NST;
-        if (!mbar_wait(v_full + s, (j / C::NST) & 1, abort, ctl, kSiteFwdMma)) break;
-        for (int x = 0; ok && x < 2; ++x) {
-          if (j >= n_x[x]) continue;
-          if (!mbar_wait(p_full + x, j & 1, abort, ctl, kSiteFwdMma)) {
+      __syncwarp();
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (leader) mma_commit(bar);
+      __syncwarp();
+    };
+    bool ok = wait_all(q_full, 0, abort, ctl, kSiteFwdMma) && wait_k(0);
+    if (ok) {
+      tc_fence_after();
+      for (int x = 0; x < 2; ++x)
+        if (n_x[x] > 0) issue_s(x, 0);
+      commit(k_empty + 0);
+    }
+    for (int j = 0; ok && j < n_max; ++j) {
+      const int s = j % C::NST;
+      if (!wait_all(v_full + s, (j / C::NST) & 1, abort, ctl, kSiteFwdMma)) break;
+      for (int x = 0; ok && x < 2; ++x) {
+        if (j >= n_x[x]) continue;
+        if (!wait_all(p_full + x, j & 1, abort, ctl, kSiteFwdMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(x, j);
+        if (j + 1 < n_x[x]) {
+          if (!wait_k(j + 1)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          issue_pv(x, j);
-          if (j + 1 < n_x[x]) {
-            if (!wait_k(j + 1)) {
-              ok = false;
-              break;
-            }
-            issue_s(x, j + 1);
-          }
+          issue_s(x, j + 1);
         }
-        if (!ok) break;
-        mma_commit(v_empty + s);
-        if (j + 1 < n_max) mma_commit(k_empty + (j + 1) % C::NST);
       }
+      if (!ok) break;
+      commit(v_empty + s);
+      if (j + 1 < n_max) commit(k_empty + (j + 1) % C::NST);
     }
     __syncwarp();
   }
