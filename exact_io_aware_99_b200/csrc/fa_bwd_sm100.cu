@@ -727,8 +727,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ launch
 
+// Heads per group, from the bytes every CTA of a head re-reads (Q and dO for
+// the dK/dV kernel, K and V for the dQ kernel: 4 N d each): a group's share
+// stays within ~64 MB of the 126 MB L2, and the groups are large enough that
+// the longest-first order ends on short CTAs (small groups start their last
+// group's long CTAs at the end and leave SMs idle).
 inline int heads_per_group(long long per_head_bytes, int BH) {
-  int g = static_cast<int>((48LL << 20) / (per_head_bytes > 0 ? per_head_bytes : 1));
+  int g = static_cast<int>((64LL << 20) / (per_head_bytes > 0 ? per_head_bytes : 1));
   return g < 1 ? 1 : (g > BH ? BH : g);
 }
 
@@ -752,7 +757,7 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   // Heads per group: a group's Q, K, V, dO (bf16, 8 N d bytes per head)
   // within ~48 MB of the 126 MB L2.
-  const int group = heads_per_group(8LL * N * D, BH);
+  const int group = heads_per_group(4LL * N * D, BH);
   const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};
   bwd_dkdv_kernel<D, CAUSAL>
