@@ -53,6 +53,7 @@ constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 #ifndef FA_FWD_POLY_EVERY
 #define FA_FWD_POLY_EVERY 0  // one column pair in this many uses the FMA-pipe exp2 (0: none)
 #endif
+constexpr int kPolyMod = FA_FWD_POLY_EVERY > 0 ? FA_FWD_POLY_EVERY : 1;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -65,12 +66,13 @@ struct Cfg {
   static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + NST * TILE;
   static constexpr int BAR_OFF = V_OFF + NST * TILE;
-  static constexpr int NBAR = 1 + 4 * NST + 6 + 8;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int SMEM = MISC_OFF + 16 + 1024;  // + slack for 1 KB alignment
+  static constexpr int NBAR = 2 + 4 * NST + 6 + 8 + 4;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
+  static constexpr int SMEM = MISC_OFF + 48 + 1024;    // + slack for 1 KB alignment
   static constexpr int KSTEPS = D / 16;
   static_assert(D % 16 == 0 && D <= 128, "head dim must be a multiple of 16, <= 128");
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(MISC_OFF % 16 == 0, "next-item responses need 16-byte alignment");
 };
 
 // Drain wait used only while aborting: ignores the abort flag, bounded by time.
@@ -91,6 +93,28 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, w);
 }
 
+// (bh, tile pair) and the key tiles each of the pair's query tiles visits
+// (0 when tile B lies past N), for work item `idx` in group-major order:
+// `group` heads at a time (their K and V stay in L2), and inside a group the
+// longest tile pairs first, head fastest.
+template <bool CAUSAL>
+__device__ __forceinline__ void decode_item(int idx, int n_t, int BH, int group, int& bh,
+                                            int& pair, int (&n_x)[2]) {
+  const int n_pair = (n_t + 1) / 2;
+  const int per_group = group * n_pair;
+  const int g = idx / per_group;
+  const int r = idx - g * per_group;
+  const int gh = min(group, BH - g * group);
+  const int t = r / gh;
+  pair = n_pair - 1 - t;
+  bh = g * group + (r - t * gh);
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int qt = 2 * pair + x;
+    n_x[x] = qt >= n_t ? 0 : (CAUSAL ? min(qt + 1, n_t) : n_t);
+  }
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -105,7 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
+  uint64_t* q_empty = bars + 1;         // Q tiles no longer read by the item's S MMAs
+  uint64_t* k_full = bars + 2;
   uint64_t* k_empty = k_full + C::NST;
   uint64_t* v_full = k_empty + C::NST;
   uint64_t* v_empty = v_full + C::NST;
@@ -117,35 +142,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   // "A's warp w finished exp(j)", tok_ba[w] "B's warp w finished exp(j)".
   uint64_t* tok_ab = o_done + 2;        // [4]
   uint64_t* tok_ba = tok_ab + 4;        // [4]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  // Next-item requests (cluster launch control), double-buffered: the
+  // producer issues the request for item i + 1 into slot (i + 1) & 1 once it
+  // has issued item i's loads; the MMA warp and the 8 softmax warps read it
+  // when they move on, and release the slot through nxt_empty.
+  uint64_t* nxt_full = tok_ba + 4;      // [2]
+  uint64_t* nxt_empty = nxt_full + 2;   // [2]
+  uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 36);
 
   const int warp = warp_id();
   const int lane = lane_id();
   const int n_t = (N + kBN - 1) / kBN;  // query tiles == key tiles
-  const int n_pair = (n_t + 1) / 2;
-  // Group-major order: `group` heads at a time (their K and V stay in L2),
-  // and inside a group the longest tile pairs first, head fastest.
-  int bh, pair;
-  {
-    const int per_group = group * n_pair;
-    const int g = static_cast<int>(blockIdx.x) / per_group;
-    const int r = static_cast<int>(blockIdx.x) - g * per_group;
-    const int gh = min(group, BH - g * group);
-    const int t = r / gh;
-    pair = n_pair - 1 - t;
-    bh = g * group + (r - t * gh);
-  }
-  const int qt[2] = {2 * pair, 2 * pair + 1};
-  // Key tiles each query tile visits (0 when tile B lies past N).
-  int n_x[2];
-#pragma unroll
-  for (int x = 0; x < 2; ++x)
-    n_x[x] = qt[x] >= n_t ? 0 : (CAUSAL ? min(qt[x] + 1, n_t) : n_t);
-  const int n_max = max(n_x[0], n_x[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
@@ -156,6 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(s_full + x, 1);
       mbar_init(p_full + x, kBM);
       mbar_init(o_done + x, 1);
+      mbar_init(nxt_full + x, 1);
+      mbar_init(nxt_empty + x, 9);  // MMA warp + 8 softmax warps
     }
     for (int w = 0; w < 4; ++w) {
       mbar_init(tok_ab + w, 1);
@@ -173,6 +188,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Work item i of this CTA: its own index first, then the CTAs it
+  // cancelled.  Consumers read the request the producer issued during item
+  // i - 1 (use (i - 1) >> 1 of slot i & 1) and release the slot.  Returns
+  // false when a wait gave up; idx < 0 means the grid has no work left.
+  auto next_item = [&](int i, int& idx, int site) -> bool {
+    if (i == 0) {
+      idx = static_cast<int>(blockIdx.x);
+      return true;
+    }
+    const int sl = i & 1;
+    if (!wait_all(nxt_full + sl, static_cast<uint32_t>((i - 1) >> 1) & 1, abort, ctl, site))
+      return false;
+    idx = clc_result_x(nxt_resp + 16 * sl);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(nxt_empty + sl);
+    return true;
+  };
+
   if (warp >= 8) {
   regs_decrease<kControlRegs>();
   if (warp == 8) {
@@ -184,40 +217,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last_k[C::NST], last_v[C::NST];
 #pragma unroll
       for (int s = 0; s < C::NST; ++s) last_k[s] = last_v[s] = -1;
-      const int nq = n_x[1] > 0 ? 2 : 1;
-      mbar_arrive_expect_tx(q_full, nq * C::TILE);
-      for (int x = 0; x < nq; ++x)
-#pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-          tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + x * C::TILE + b * C::BLK, b * 64,
-                      qt[x] * kBM, bh);
-      for (int j = 0; j < n_max; ++j) {
-        const int s = j % C::NST;
-        const uint32_t u = static_cast<uint32_t>(j / C::NST);
-        if (j >= C::NST && !mbar_wait(k_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer))
+      int q_issued = 0;           // Q loads issued (one per item)
+      int nxt_pending = -1;       // slot of a request in flight
+      uint32_t nxt_pending_par = 0;
+      uint32_t kv = 0;            // K/V ring uses so far
+      int idx = static_cast<int>(blockIdx.x);
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        if (i > 0) {
+          const int sl = i & 1;
+          if (!mbar_wait(nxt_full + sl, static_cast<uint32_t>((i - 1) >> 1) & 1, abort, ctl,
+                         kSiteFwdProducer))
+            break;
+          nxt_pending = -1;
+          idx = clc_result_x(nxt_resp + 16 * sl);
+          if (idx < 0) break;
+        }
+        int bh, pair, n_x[2];
+        decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+        const int n_max = max(n_x[0], n_x[1]);
+        // Q of this item replaces the previous item's once its S MMAs are done.
+        if (i > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(i - 1) & 1, abort, ctl,
+                                kSiteFwdProducer))
           break;
-        mbar_arrive_expect_tx(k_full + s, C::TILE);
+        const int nq = n_x[1] > 0 ? 2 : 1;
+        mbar_arrive_expect_tx(q_full, nq * C::TILE);
+        for (int x = 0; x < nq; ++x)
 #pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-          tma_load_3d(&tm_k, k_full + s, smem + C::K_OFF + s * C::TILE + b * C::BLK, b * 64,
-                      j * kBN, bh);
-        last_k[s] = static_cast<int>(u);
-        if (j >= C::NST && !mbar_wait(v_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer))
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + x * C::TILE + b * C::BLK, b * 64,
+                        (2 * pair + x) * kBM, bh);
+        q_issued = i + 1;
+        for (int j = 0; j < n_max; ++j, ++kv) {
+          const int s = static_cast<int>(kv % C::NST);
+          const uint32_t u = kv / C::NST;
+          if (kv >= C::NST && !mbar_wait(k_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(k_full + s, C::TILE);
+#pragma unroll
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_3d(&tm_k, k_full + s, smem + C::K_OFF + s * C::TILE + b * C::BLK, b * 64,
+                        j * kBN, bh);
+          last_k[s] = static_cast<int>(u);
+          if (kv >= C::NST && !mbar_wait(v_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(v_full + s, C::TILE);
+#pragma unroll
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_3d(&tm_v, v_full + s, smem + C::V_OFF + s * C::TILE + b * C::BLK, b * 64,
+                        j * kBN, bh);
+          last_v[s] = static_cast<int>(u);
+        }
+        if (!ok) break;
+        // Ask for the next item now, while this one's MMAs and softmax run.
+        const int sl1 = (i + 1) & 1;
+        const uint32_t u1 = static_cast<uint32_t>(i >> 1);
+        if (u1 > 0 && !mbar_wait(nxt_empty + sl1, (u1 - 1) & 1, abort, ctl, kSiteFwdProducer))
           break;
-        mbar_arrive_expect_tx(v_full + s, C::TILE);
-#pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-          tma_load_3d(&tm_v, v_full + s, smem + C::V_OFF + s * C::TILE + b * C::BLK, b * 64,
-                      j * kBN, bh);
-        last_v[s] = static_cast<int>(u);
+        mbar_arrive_expect_tx(nxt_full + sl1, 16);
+        clc_try_cancel(nxt_resp + 16 * sl1, nxt_full + sl1);
+        nxt_pending = sl1;
+        nxt_pending_par = u1 & 1;
       }
       if (*abort) {
-        // Let every copy this CTA started land before shared memory is released.
-        drain_wait(q_full, 0, ctl);
+        // Let every copy and request this CTA started land before shared
+        // memory is released.
+        if (q_issued > 0) drain_wait(q_full, static_cast<uint32_t>(q_issued - 1) & 1, ctl);
         for (int s = 0; s < C::NST; ++s) {
           if (last_k[s] >= 0) drain_wait(k_full + s, last_k[s] & 1, ctl);
           if (last_v[s] >= 0) drain_wait(v_full + s, last_v[s] & 1, ctl);
         }
+        if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
       }
     }
     __syncwarp();
@@ -228,22 +302,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool leader = elect_one();
     constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, 0, 0);
     constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, 0, 1);
-    int k_seen = -1;  // highest key tile whose k_full wait has been done
-    auto wait_k = [&](int jj) -> bool {
-      if (jj <= k_seen) return true;
-      if (!wait_all(k_full + jj % C::NST, (jj / C::NST) & 1, abort, ctl, kSiteFwdMma))
-        return false;
-      k_seen = jj;
-      tc_fence_after();
-      return true;
-    };
     const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);       // K-major
     const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);       // K-major
     const SDesc v_desc = sdesc(sbase + C::V_OFF, C::BLK, 1024);   // MN-major
-    auto issue_s = [&](int x, int jj) {  // S_x = Q_x K_jj^T
+    uint32_t kv_base = 0;            // K/V ring uses before this item
+    uint32_t p_base[2] = {0u, 0u};   // p_full phases consumed before this item
+    int k_seen = -1;                 // highest ring use whose k_full wait was done
+    auto wait_k = [&](int r) -> bool {  // ring use r
+      if (r <= k_seen) return true;
+      if (!wait_all(k_full + r % C::NST, static_cast<uint32_t>(r / C::NST) & 1, abort, ctl,
+                    kSiteFwdMma))
+        return false;
+      k_seen = r;
+      tc_fence_after();
+      return true;
+    };
+    auto issue_s = [&](int x, int r) {  // S_x = Q_x K^T, K in ring use r
       if (leader) {
         const SDesc qd = q_desc + x * C::TILE;
-        const SDesc kd = k_desc + (jj % C::NST) * C::TILE;
+        const SDesc kd = k_desc + (r % C::NST) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
@@ -253,13 +330,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    auto issue_pv = [&](int x, int jj) {  // O_x += P_x V_jj, P_x from TMEM
+    auto issue_pv = [&](int x, int r, bool first) {  // O_x (+)= P_x V, P_x from TMEM
       if (leader) {
-        const SDesc vd = v_desc + (jj % C::NST) * C::TILE;
+        const SDesc vd = v_desc + (r % C::NST) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_ts(tmem + 256 + x * kBN, tmem + x * kBN + kk * 8, vd + kk * 16 * 128, kIdescPV,
-                 (jj > 0 || kk > 0) ? 1u : 0u);
+                 (!first || kk > 0) ? 1u : 0u);
         mma_commit(o_done + x);
       }
       __syncwarp();
@@ -268,35 +345,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) mma_commit(bar);
       __syncwarp();
     };
-    bool ok = wait_all(q_full, 0, abort, ctl, kSiteFwdMma) && wait_k(0);
-    if (ok) {
+    bool ok = true;
+    int idx = 0;
+    for (int i = 0; ok; ++i) {
+      if (!next_item(i, idx, kSiteFwdMma)) break;
+      if (idx < 0) break;
+      int bh, pair, n_x[2];
+      decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+      const int n_max = max(n_x[0], n_x[1]);
+      const int r0 = static_cast<int>(kv_base);
+      ok = wait_all(q_full, static_cast<uint32_t>(i) & 1, abort, ctl, kSiteFwdMma) && wait_k(r0);
+      if (!ok) break;
       tc_fence_after();
       for (int x = 0; x < 2; ++x)
-        if (n_x[x] > 0) issue_s(x, 0);
-      commit(k_empty + 0);
-    }
-    for (int j = 0; ok && j < n_max; ++j) {
-      const int s = j % C::NST;
-      if (!wait_all(v_full + s, (j / C::NST) & 1, abort, ctl, kSiteFwdMma)) break;
-      for (int x = 0; ok && x < 2; ++x) {
-        if (j >= n_x[x]) continue;
-        if (!wait_all(p_full + x, j & 1, abort, ctl, kSiteFwdMma)) {
+        if (n_x[x] > 0) issue_s(x, r0);
+      commit(k_empty + r0 % C::NST);
+      if (n_max == 1) commit(q_empty);
+      for (int j = 0; ok && j < n_max; ++j) {
+        const int r = r0 + j;
+        if (!wait_all(v_full + r % C::NST, static_cast<uint32_t>(r / C::NST) & 1, abort, ctl,
+                      kSiteFwdMma)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        issue_pv(x, j);
-        if (j + 1 < n_x[x]) {
-          if (!wait_k(j + 1)) {
+        for (int x = 0; ok && x < 2; ++x) {
+          if (j >= n_x[x]) continue;
+          if (!wait_all(p_full + x, (p_base[x] + j) & 1, abort, ctl, kSiteFwdMma)) {
             ok = false;
             break;
           }
-          issue_s(x, j + 1);
+          tc_fence_after();
+          issue_pv(x, r, j == 0);
+          if (j + 1 < n_x[x]) {
+            if (!wait_k(r + 1)) {
+              ok = false;
+              break;
+            }
+            issue_s(x, r + 1);
+          }
         }
+        if (!ok) break;
+        commit(v_empty + r % C::NST);
+        if (j + 1 < n_max) commit(k_empty + (r + 1) % C::NST);
+        if (j + 2 == n_max) commit(q_empty);  // the item's last S MMAs are issued
       }
-      if (!ok) break;
-      commit(v_empty + s);
-      if (j + 1 < n_max) commit(k_empty + (j + 1) % C::NST);
+      kv_base += static_cast<uint32_t>(n_max);
+      p_base[0] += static_cast<uint32_t>(n_x[0]);
+      p_base[1] += static_cast<uint32_t>(n_x[1]);
     }
     __syncwarp();
   }
@@ -305,147 +400,168 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------- softmax (warps 0-3: A, 4-7: B)
     const int x = warp >> 2;
     const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int wq = warp & 3;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t col_s = x * kBN;
     const uint32_t col_o = 256 + x * kBN;
-    const int n_kv = n_x[x];
-    const int q_idx = qt[x] * kBM + r;
-    float m = -INFINITY;  // reference max, base-2 scaled units
-    float l = 0.f;
+    // Phases of this tile's barriers consumed before the current item.
+    uint32_t s_base = 0, tab_base = 0, tba_base = 0;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!wait_all(s_full + x, j & 1, abort, ctl, kSiteFwdSoftmax)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[kBN];
-      {
-        uint32_t t0[32], t1[32];
-        tmem_ld32(lane_base + col_s + 0, t0);
-        tmem_ld32(lane_base + col_s + 32, t1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          s[c] = __uint_as_float(t0[c]);
-          s[32 + c] = __uint_as_float(t1[c]);
+    int idx = 0;
+    for (int i = 0; ok; ++i) {
+      if (!next_item(i, idx, kSiteFwdSoftmax)) break;
+      if (idx < 0) break;
+      int bh, pair, n_x[2];
+      decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+      const int n_kv = n_x[x];
+      const int q_idx = (2 * pair + x) * kBM + r;
+      float m = -INFINITY;  // reference max, base-2 scaled units
+      float l = 0.f;
+      for (int j = 0; j < n_kv; ++j) {
+        if (!wait_all(s_full + x, (s_base + j) & 1, abort, ctl, kSiteFwdSoftmax)) {
+          ok = false;
+          break;
         }
-        tmem_ld32(lane_base + col_s + 64, t0);
-        tmem_ld32(lane_base + col_s + 96, t1);
-        tmem_wait_ld();
+        tc_fence_after();
+        float s[kBN];
+        {
+          uint32_t t0[32], t1[32];
+          tmem_ld32(lane_base + col_s + 0, t0);
+          tmem_ld32(lane_base + col_s + 32, t1);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          s[64 + c] = __uint_as_float(t0[c]);
-          s[96 + c] = __uint_as_float(t1[c]);
+          for (int c = 0; c < 32; ++c) {
+            s[c] = __uint_as_float(t0[c]);
+            s[32 + c] = __uint_as_float(t1[c]);
+          }
+          tmem_ld32(lane_base + col_s + 64, t0);
+          tmem_ld32(lane_base + col_s + 96, t1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            s[64 + c] = __uint_as_float(t0[c]);
+            s[96 + c] = __uint_as_float(t1[c]);
+          }
         }
-      }
-      const int kv0 = j * kBN;
-      const bool diag = CAUSAL && (j == n_kv - 1);
-      const bool masked = diag || kv0 + kBN > N;
-      const int lim = masked ? min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN) : kBN;
-      if (masked) {
+        const int kv0 = j * kBN;
+        const bool diag = CAUSAL && (j == n_kv - 1);
+        const bool masked = diag || kv0 + kBN > N;
+        const int lim = masked ? min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN) : kBN;
+        if (masked) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c >= lim) s[c] = -INFINITY;
-      }
-      float mx4[4] = {s[0], s[1], s[2], s[3]};
+          for (int c = 0; c < kBN; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
+        float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int c = 4; c < kBN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      const float m_cand = fmaxf(m, mx * scale_log2);
-      const bool grow = m_cand > m + kRescaleLog2;  // true on the first tile
-      const float alpha = grow ? ex2(m - m_cand) : 1.f;
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_x += P_x(j-1) V completed before S_x(j) (same MMA thread, in
-        // order), so O_x can be rescaled now.
+        for (int c = 4; c < kBN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float m_cand = fmaxf(m, mx * scale_log2);
+        const bool grow = m_cand > m + kRescaleLog2;  // true on the first tile
+        const float alpha = grow ? ex2(m - m_cand) : 1.f;
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O_x += P_x(j-1) V completed before S_x(j) (same MMA thread, in
+          // order), so O_x can be rescaled now.
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o16[16];
+            tmem_ld16(lane_base + col_o + c * 16, o16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
+            tmem_st16(lane_base + col_o + c * 16, o16);
+          }
+        }
+        if (grow) {
+          l *= alpha;
+          m = m_cand;
+        }
+        // The two tiles' warps on one sub-partition take turns on the MUFU:
+        // A(0), B(0), A(1), B(1), ...  (only while both tiles still run).
+        if (x == 0 ? (j >= 1 && j - 1 < n_x[1]) : (j < n_x[0])) {
+          uint64_t* tok = x == 0 ? tok_ba + wq : tok_ab + wq;
+          const uint32_t par = x == 0 ? (tba_base + j - 1) & 1 : (tab_base + j) & 1;
+          if (!wait_all(tok, par, abort, ctl, kSiteFwdSoftmax)) {
+            ok = false;
+            break;
+          }
+        }
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        const float2 sc2 = make_float2(scale_log2, scale_log2);
+        const float2 nm2 = make_float2(neg_m, neg_m);
+        // One column pair in FA_FWD_POLY_EVERY goes to the FMA-pipe exp2, the
+        // rest to the special-function unit, so the two units share the work.
+        float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+        uint32_t pk[kBN / 2];
+#pragma unroll
+        for (int c = 0; c < kBN / 2; ++c) {
+          const float2 xx = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+          float2 p;
+          if (FA_FWD_POLY_EVERY > 0 && c % kPolyMod == kPolyMod - 1) {
+            p = exp2_fma2(xx);
+            if (masked) {
+              if (2 * c >= lim) p.x = 0.f;
+              if (2 * c + 1 >= lim) p.y = 0.f;
+            }
+          } else {
+            p = make_float2(ex2(xx.x), ex2(xx.y));
+          }
+          rs2[c & 3] = __fadd2_rn(rs2[c & 3], p);
+          pk[c] = pack_bf16(p.x, p.y);
+        }
+        const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+        const float rs = rsa.x + rsa.y;
+        __syncwarp();
+        if (lane == 0 && (x == 0 ? (j < n_x[1]) : (j + 1 < n_x[0])))
+          mbar_arrive(x == 0 ? tok_ab + wq : tok_ba + wq);
+        l += rs;
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+          tmem_st32(lane_base + col_s + 0, lo);
+          tmem_st32(lane_base + col_s + 32, hi);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + x);
+      }
+      // -------------------------------------------------------- epilogue
+      // o_done completes once per P V of this tile; its last phase of this
+      // item is s_base + n_kv - 1.
+      if (ok && n_kv > 0 &&
+          wait_all(o_done + x, (s_base + n_kv - 1) & 1, abort, ctl, kSiteFwdEpilogue)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool valid = q_idx < N;
+        uint4* orow = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
           uint32_t o16[16];
           tmem_ld16(lane_base + col_o + c * 16, o16);
           tmem_wait_ld();
+          uint32_t pkd[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
-          tmem_st16(lane_base + col_o + c * 16, o16);
-        }
-      }
-      if (grow) {
-        l *= alpha;
-        m = m_cand;
-      }
-      // The two tiles' warps on one sub-partition take turns on the MUFU:
-      // A(0), B(0), A(1), B(1), ...  (only while both tiles still run).
-      const int wq = warp & 3;
-      if (x == 0 ? (j >= 1 && j - 1 < n_x[1]) : (j < n_x[0])) {
-        uint64_t* tok = x == 0 ? tok_ba + wq : tok_ab + wq;
-        const uint32_t par = static_cast<uint32_t>(x == 0 ? j - 1 : j) & 1;
-        if (!wait_all(tok, par, abort, ctl, kSiteFwdSoftmax)) {
-          ok = false;
-          break;
-        }
-      }
-      const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      const float2 sc2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(neg_m, neg_m);
-      // One column pair in FA_FWD_POLY_EVERY goes to the FMA-pipe exp2, the
-      // rest to the special-function unit, so the two units share the work.
-      float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                       make_float2(0.f, 0.f)};
-      uint32_t pk[kBN / 2];
-#pragma unroll
-      for (int c = 0; c < kBN / 2; ++c) {
-        const float2 xx = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
-        float2 p;
-        if (FA_FWD_POLY_EVERY > 0 && c % FA_FWD_POLY_EVERY == FA_FWD_POLY_EVERY - 1) {
-          p = exp2_fma2(xx);
-          if (masked) {
-            if (2 * c >= lim) p.x = 0.f;
-            if (2 * c + 1 >= lim) p.y = 0.f;
+          for (int e = 0; e < 8; ++e)
+            pkd[e] = pack_bf16(__uint_as_float(o16[2 * e]) * inv_l,
+                               __uint_as_float(o16[2 * e + 1]) * inv_l);
+          if (valid) {
+            orow[2 * c] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+            orow[2 * c + 1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
           }
-        } else {
-          p = make_float2(ex2(xx.x), ex2(xx.y));
         }
-        rs2[c & 3] = __fadd2_rn(rs2[c & 3], p);
-        pk[c] = pack_bf16(p.x, p.y);
+        if (valid)
+          lse[static_cast<size_t>(bh) * N + q_idx] = (m + __log2f(l)) * 0.69314718055994531f;
+        // The next item's first P V (accumulate off) overwrites O_x only
+        // after this warpgroup's next P, so the loads above are complete.
+        tc_fence_before();
+      } else if (ok && n_kv > 0) {
+        ok = false;
       }
-      const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
-      const float rs = rsa.x + rsa.y;
-      __syncwarp();
-      if (lane == 0 && (x == 0 ? (j < n_x[1]) : (j + 1 < n_x[0])))
-        mbar_arrive(x == 0 ? tok_ab + wq : tok_ba + wq);
-      l += rs;
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-        tmem_st32(lane_base + col_s + 0, lo);
-        tmem_st32(lane_base + col_s + 32, hi);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full + x);
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok && n_kv > 0 && wait_all(o_done + x, (n_kv - 1) & 1, abort, ctl, kSiteFwdEpilogue)) {
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      const bool valid = q_idx < N;
-      uint4* orow = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t o16[16];
-        tmem_ld16(lane_base + col_o + c * 16, o16);
-        tmem_wait_ld();
-        uint32_t pkd[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          pkd[e] = pack_bf16(__uint_as_float(o16[2 * e]) * inv_l,
-                             __uint_as_float(o16[2 * e + 1]) * inv_l);
-        if (valid) {
-          orow[2 * c] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
-          orow[2 * c + 1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
-        }
-      }
-      if (valid)
-        lse[static_cast<size_t>(bh) * N + q_idx] = (m + __log2f(l)) * 0.69314718055994531f;
+      s_base += static_cast<uint32_t>(n_kv);
+      tab_base += static_cast<uint32_t>(min(n_x[0], n_x[1]));
+      tba_base += static_cast<uint32_t>(max(0, min(n_x[0] - 1, n_x[1])));
     }
   }
 

@@ -102,6 +102,39 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* m, uint64_t* bar,
       : "memory");
 }
 
+// ------------------------------------------------- cluster launch control
+
+// Ask the hardware to cancel the launch of a CTA of this grid that has not
+// started yet (sm_100 cluster launch control).  The 16-byte response lands in
+// shared memory at `resp16` (16-byte aligned) as transaction bytes on `bar`;
+// the caller has armed `bar` with mbar_arrive_expect_tx(bar, 16).  A CTA
+// whose request succeeds must run the cancelled CTA's work itself, which
+// makes a grid of ordinary CTAs behave like persistent ones that take work
+// in launch order.
+__device__ __forceinline__ void clc_try_cancel(void* resp16, uint64_t* bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128"
+      " [%0], [%1];" ::"r"(smem_u32(resp16)),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+// blockIdx.x of the CTA a completed request cancelled, or -1 when the grid
+// had no CTA left to cancel.
+__device__ __forceinline__ int clc_result_x(const void* resp16) {
+  uint32_t canceled, x = 0;
+  asm volatile(
+      "{\n\t.reg .b128 rsp;\n\t.reg .pred p;\n\t"
+      "ld.shared.b128 rsp, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, rsp;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, rsp;\n\t}"
+      : "=r"(canceled), "+r"(x)
+      : "r"(smem_u32(resp16))
+      : "memory");
+  return canceled ? static_cast<int>(x) : -1;
+}
+
 // Contiguous (untiled) bulk copy global -> shared, completion as transaction
 // bytes on `bar`.  Both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
