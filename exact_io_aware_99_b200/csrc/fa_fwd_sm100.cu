@@ -11,12 +11,17 @@
 // P never leave the SM: S lives in tensor memory (TMEM), P is written back
 // over S as bf16 and fed to the second MMA straight from TMEM.
 //
-// B200 design: one CTA per pair of 128-row query tiles (A = 2p, B = 2p+1)
-// of one head, 12 warps (warps 10-11 idle; the third warpgroup gives its
-// registers to the two softmax warpgroups):
-//   warp 8      TMA producer: both Q tiles once, then K_j and V_j into
+// B200 design: a work item is a pair of 128-row query tiles (A = 2p,
+// B = 2p+1) of one head; the grid has one CTA per item, and a running CTA
+// takes further items by cancelling CTAs that have not started yet (cluster
+// launch control), so one CTA per SM works through items in launch order and
+// the rings, barriers and TMEM carry over from one item to the next.
+// 12 warps (warps 10-11 idle; the third warpgroup gives its registers to the
+// two softmax warpgroups):
+//   warp 8      TMA producer: both Q tiles of an item, then K_j and V_j into
 //               separate shared-memory rings; each K/V tile serves both Q
-//               tiles (half the K/V traffic per FLOP of a one-tile CTA).
+//               tiles (half the K/V traffic per FLOP of a one-tile CTA).  It
+//               requests the next item once the current item's loads are out.
 //   warp 9      TMEM allocator and MMA issuer (one elected lane), alternating
 //               between the tiles: O_A += P_A V_j, S_A = Q_A K_{j+1}^T,
 //               O_B += P_B V_j, S_B = Q_B K_{j+1}^T, so the tensor core works
@@ -66,7 +71,7 @@ struct Cfg {
   static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + NST * TILE;
   static constexpr int BAR_OFF = V_OFF + NST * TILE;
-  static constexpr int NBAR = 2 + 4 * NST + 6 + 8 + 4;
+  static constexpr int NBAR = 2 + 4 * NST + 6 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
   static constexpr int SMEM = MISC_OFF + 48 + 1024;    // + slack for 1 KB alignment
   static constexpr int KSTEPS = D / 16;
@@ -137,16 +142,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = v_empty + C::NST;  // [2] per tile
   uint64_t* p_full = s_full + 2;        // [2] per tile
   uint64_t* o_done = p_full + 2;        // [2] per tile
-  // Exponential-phase tokens between the two warps that share an SM
-  // sub-partition (warp w of tile A, warp w + 4 of tile B): tok_ab[w] says
-  // "A's warp w finished exp(j)", tok_ba[w] "B's warp w finished exp(j)".
-  uint64_t* tok_ab = o_done + 2;        // [4]
-  uint64_t* tok_ba = tok_ab + 4;        // [4]
   // Next-item requests (cluster launch control), double-buffered: the
   // producer issues the request for item i + 1 into slot (i + 1) & 1 once it
   // has issued item i's loads; the MMA warp and the 8 softmax warps read it
   // when they move on, and release the slot through nxt_empty.
-  uint64_t* nxt_full = tok_ba + 4;      // [2]
+  uint64_t* nxt_full = o_done + 2;      // [2]
   uint64_t* nxt_empty = nxt_full + 2;   // [2]
   uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
@@ -171,10 +171,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(o_done + x, 1);
       mbar_init(nxt_full + x, 1);
       mbar_init(nxt_empty + x, 9);  // MMA warp + 8 softmax warps
-    }
-    for (int w = 0; w < 4; ++w) {
-      mbar_init(tok_ab + w, 1);
-      mbar_init(tok_ba + w, 1);
     }
     *abort = 0;
     fence_barrier_init();
@@ -400,12 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------- softmax (warps 0-3: A, 4-7: B)
     const int x = warp >> 2;
     const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
-    const int wq = warp & 3;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t col_s = x * kBN;
     const uint32_t col_o = 256 + x * kBN;
-    // Phases of this tile's barriers consumed before the current item.
-    uint32_t s_base = 0, tab_base = 0, tba_base = 0;
+    uint32_t s_base = 0;  // s_full / o_done phases of this tile before the current item
     bool ok = true;
     int idx = 0;
     for (int i = 0; ok; ++i) {
@@ -477,16 +471,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
           m = m_cand;
         }
-        // The two tiles' warps on one sub-partition take turns on the MUFU:
-        // A(0), B(0), A(1), B(1), ...  (only while both tiles still run).
-        if (x == 0 ? (j >= 1 && j - 1 < n_x[1]) : (j < n_x[0])) {
-          uint64_t* tok = x == 0 ? tok_ba + wq : tok_ab + wq;
-          const uint32_t par = x == 0 ? (tba_base + j - 1) & 1 : (tab_base + j) & 1;
-          if (!wait_all(tok, par, abort, ctl, kSiteFwdSoftmax)) {
-            ok = false;
-            break;
-          }
-        }
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
         const float2 sc2 = make_float2(scale_log2, scale_log2);
         const float2 nm2 = make_float2(neg_m, neg_m);
@@ -513,9 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
         const float rs = rsa.x + rsa.y;
-        __syncwarp();
-        if (lane == 0 && (x == 0 ? (j < n_x[1]) : (j + 1 < n_x[0])))
-          mbar_arrive(x == 0 ? tok_ab + wq : tok_ba + wq);
         l += rs;
         {
           uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
@@ -560,8 +541,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
       }
       s_base += static_cast<uint32_t>(n_kv);
-      tab_base += static_cast<uint32_t>(min(n_x[0], n_x[1]));
-      tba_base += static_cast<uint32_t>(max(0, min(n_x[0] - 1, n_x[1])));
     }
   }
 
