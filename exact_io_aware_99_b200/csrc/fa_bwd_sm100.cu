@@ -23,8 +23,10 @@
 //        dS^T = P^T o (dP^T - D) into already-read columns of B (bf16)
 //      dV += P^T dO_i     (TS, P^T from TMEM)  -> cols [256,256+d)
 //      dK += dS^T Q_i     (TS, dS^T from TMEM) -> cols [384,384+d)
-//    issued as S_0, dP_0, dV_0, S_1, dK_0, dP_1, dV_1, S_2, dK_1, ... so the
-//    softmax forms P_{i+1} while the tensor core runs dK_i and dP_{i+1}.
+//    issued as S_0, dP_0, [P_0] dV_0, S_1, [dS_0] dK_0, dP_1, [P_1] dV_1,
+//    S_2, [dS_1] dK_1, ... : S_{i+1} goes in right behind dV_i (which
+//    releases P_i's columns), so it is ready when the softmax finishes dS_i,
+//    and the softmax forms P_{i+1} while the tensor core runs dK_i, dP_{i+1}.
 //  dQ kernel -- one CTA per (head, 128-query tile Q_i), looping over the key
 //  tiles K_j it sees.  Per key tile:
 //      S  = Q_i K_j^T     (SS)  -> TMEM S buffer j%2 (double-buffered)
@@ -48,6 +50,15 @@ namespace fa {
 namespace bwd {
 
 constexpr int kT = 128;  // rows of every tile (keys or queries)
+// Issue-order switches (both on; off gives the older, slower orders):
+// dK/dV kernel: S_{i+1} right after dV_i instead of after dS_i;
+// dQ kernel: dP_{j+1} ahead of dQ_j.
+#ifndef FA_BWD_EARLY_S
+#define FA_BWD_EARLY_S 1
+#endif
+#ifndef FA_BWD_EARLY_DP
+#define FA_BWD_EARLY_DP 1
+#endif
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 
@@ -293,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       // S^T_{i+1} overwrites P^T_i in A: issued after dV_i (same thread, in
-      // order) and after the softmax finished reading P^T_i (ds_full).
+      // order); the softmax is done with A once it signalled p_full.
       // dP^T_{i+1} overwrites dS^T_i in B: issued after dK_i, in order.
       bool ok = wait_all(kv_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
       for (int it = 0; ok && it < n_iter; ++it) {
@@ -312,9 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                    (it > 0 || kk > 0) ? 1u : 0u);
         }
         __syncwarp();
+        if (FA_BWD_EARLY_S && it + 1 < n_iter && !issue_s(it + 1)) break;
         if (!wait_all(ds_full, it & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
-        if (it + 1 < n_iter && !issue_s(it + 1)) break;
+        if (!FA_BWD_EARLY_S && it + 1 < n_iter && !issue_s(it + 1)) break;
         // dK += dS^T Q_i: dS^T k-step kk at column 128 + 64*(kk/4) + 8*(kk%4).
         if (leader) {
 #pragma unroll
@@ -630,16 +642,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         return true;
       };
-      // Order: S_0, dP_0, S_1, [dS_0] dQ_0, dP_1, S_2, [dS_1] dQ_1, ... so the
-      // tensor core computes S_{j+1} while the softmax warps form dS_j.  S_{j+2}
-      // reuses S_j's buffer after dQ_j has read dS_j (same thread, in order)
-      // and the softmax released it (ds_full waited); dP_{j+1} likewise.
+      // Order: S_0, dP_0, S_1, [dS_0] dP_1, dQ_0, S_2, [dS_1] dP_2, dQ_1, ...
+      // so the tensor core computes S_{j+1} while the softmax warps form dS_j,
+      // and dP_{j+1} is ready soon after.  S_{j+2} reuses S_j's buffer after
+      // dQ_j has read dS_j (same thread, in order) and the softmax released it
+      // (ds_full waited); dP_{j+1} overwrites dP_j once ds_full(j) says the
+      // softmax has read it.
       bool ok = wait_all(q_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
       if (ok && n_kv > 1) ok = issue_s(1);
       for (int jj = 0; ok && jj < n_kv; ++jj) {
         const int s = jj % C::NK;
         if (!wait_all(ds_full + (jj & 1), (jj >> 1) & 1, abort, ctl, kSiteBwdMma)) break;
         tc_fence_after();
+        if (FA_BWD_EARLY_DP && jj + 1 < n_kv && !issue_dp(jj + 1)) break;
         // dQ += dS_jj K_jj: key k-step kk (16 keys) of dS at column
         // 64*(kk/4) + 8*(kk%4) of the S buffer.
         if (leader) {
@@ -652,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(k_empty + s);
         }
         __syncwarp();
-        if (jj + 1 < n_kv && !issue_dp(jj + 1)) break;
+        if (!FA_BWD_EARLY_DP && jj + 1 < n_kv && !issue_dp(jj + 1)) break;
         if (jj + 2 < n_kv && !issue_s(jj + 2)) break;
       }
       if (leader) mma_commit(dq_done);
