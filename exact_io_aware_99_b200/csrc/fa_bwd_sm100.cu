@@ -39,8 +39,11 @@
 // Warp roles (both kernels, 10 warps): warps 0-3 and 4-7 are two softmax
 // warpgroups splitting the 128 columns of every tile in halves (one thread
 // per TMEM lane), warp 8 is the TMA producer, warp 9 the TMEM allocator and
-// MMA issuer (one elected lane).  CTAs run group-major (a few heads at a
-// time, so their operands stay in L2), longest-first inside a group.
+// MMA issuer (one elected lane).  Work items run group-major (a few heads at
+// a time, so their operands stay in L2), longest-first inside a group; the
+// grid has one CTA per item and a running CTA takes further items by
+// cancelling CTAs that have not started (cluster launch control), so the
+// pipelines, barriers and TMEM carry over from item to item.
 #include <cuda_bf16.h>
 
 #include "fa_internal.h"
@@ -59,6 +62,11 @@ constexpr int kT = 128;  // rows of every tile (keys or queries)
 #ifndef FA_BWD_EARLY_DP
 #define FA_BWD_EARLY_DP 1
 #endif
+// dK/dV kernel: one column pair in this many takes the FMA-pipe exp2 (0: none).
+#ifndef FA_BWD_POLY_EVERY
+#define FA_BWD_POLY_EVERY 6
+#endif
+constexpr int kBwdPolyMod = FA_BWD_POLY_EVERY > 0 ? FA_BWD_POLY_EVERY : 1;
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 
@@ -89,12 +97,13 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, w);
 }
 
-// (head, tile) of this CTA in group-major order: `group` heads at a time;
-// inside a group tile index t ascending, head fastest.
-__device__ __forceinline__ void group_major(int n_tiles, int BH, int group, int& bh, int& t) {
+// (head, tile) of work item idx in group-major order: `group` heads at a
+// time; inside a group tile index t ascending, head fastest.
+__device__ __forceinline__ void group_major(int idx, int n_tiles, int BH, int group, int& bh,
+                                            int& t) {
   const int per_group = group * n_tiles;
-  const int g = static_cast<int>(blockIdx.x) / per_group;
-  const int r = static_cast<int>(blockIdx.x) - g * per_group;
+  const int g = idx / per_group;
+  const int r = idx - g * per_group;
   const int gh = min(group, BH - g * group);
   t = r / gh;
   bh = g * group + (r - t * gh);
@@ -138,9 +147,10 @@ struct KvCfg : Shape<D> {
   // [2] stages of the query tile's LSE2 (512 B) then D (512 B)
   static constexpr int VEC_OFF = DO_OFF + 2 * S::TILE;
   static constexpr int BAR_OFF = VEC_OFF + 2 * 1024;
-  static constexpr int NBAR = 16;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int SMEM = MISC_OFF + 16 + 1024;
+  static constexpr int NBAR = 18;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
+  static constexpr int SMEM = MISC_OFF + 48 + 1024;
+  static_assert(MISC_OFF % 16 == 0, "next-item responses need 16-byte alignment");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -174,25 +184,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* dp_full = bars + 8;
   uint64_t* p_full = bars + 9;     // both softmax warpgroups wrote P^T
   uint64_t* ds_full = bars + 10;   // both wrote dS^T (and are done with S^T, dP^T)
-  uint64_t* kv_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  uint64_t* kv_done = bars + 11;   // the item's last dK: accumulators final
+  uint64_t* kv_empty = bars + 12;  // the item's S^T and dP^T MMAs are done with K_j, V_j
+  uint64_t* nxt_full = bars + 13;  // [2] next-item requests
+  uint64_t* nxt_empty = bars + 15; // [2]
+  uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 36);
 
   const int warp = warp_id();
   const int lane = lane_id();
   const int n_t = (N + kT - 1) / kT;
   const int Np = n_t * kT;
-  int bh, j;
-  group_major(n_t, BH, group, bh, j);  // j = 0 first: most query tiles when causal
-  const int i_start = CAUSAL ? j : 0;
-  const int n_iter = n_t - i_start;
+  // Key tile j and the query tiles [i_start, n_t) that see it, for work item
+  // idx (group-major; j = 0 first: most query tiles when causal).
+  auto decode = [&](int idx, int& bh, int& j, int& i_start, int& n_iter) {
+    group_major(idx, n_t, BH, group, bh, j);
+    i_start = CAUSAL ? j : 0;
+    n_iter = n_t - i_start;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(q_full + s, 1);
       mbar_init(do_full + s, 1);
       mbar_init(qdo_empty + s, 1);
+      mbar_init(nxt_full + s, 1);
+      mbar_init(nxt_empty + s, 9);  // MMA warp + 8 softmax warps
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -210,6 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  auto next_item = [&](int it, int& idx, int site) -> bool {
+    return next_work_item(it, idx, nxt_full, nxt_empty, nxt_resp, abort, ctl, site);
+  };
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -219,101 +242,153 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
       int last[2] = {-1, -1};
-      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
-#pragma unroll
-      for (int b = 0; b < C::NB; ++b) {
-        tma_load_3d(&tm_k, kv_full, smem + C::K_OFF + b * C::BLK, b * 64, j * kT, bh);
-        tma_load_3d(&tm_v, kv_full, smem + C::V_OFF + b * C::BLK, b * 64, j * kT, bh);
-      }
-      for (int it = 0; it < n_iter; ++it) {
-        const int st = it & 1;
-        const uint32_t u = static_cast<uint32_t>(it >> 1);
-        if (it >= 2 && !mbar_wait(qdo_empty + st, (u - 1) & 1, abort, ctl, kSiteBwdProducer))
+      int kv_issued = 0;
+      int nxt_pending = -1;
+      uint32_t nxt_pending_par = 0;
+      uint32_t qr = 0;  // query tiles streamed so far (ring uses)
+      int idx = static_cast<int>(blockIdx.x);
+      bool ok = true;
+      for (int w = 0; ok; ++w) {
+        if (w > 0) {
+          if (!producer_take_item(w, idx, nxt_full, nxt_resp, abort, ctl, kSiteBwdProducer))
+            break;
+          nxt_pending = -1;
+          if (idx < 0) break;
+        }
+        int bh, j, i_start, n_iter;
+        decode(idx, bh, j, i_start, n_iter);
+        if (w > 0 &&
+            !mbar_wait(kv_empty, static_cast<uint32_t>(w - 1) & 1, abort, ctl, kSiteBwdProducer))
           break;
-        const int y = (i_start + it) * kT;
-        mbar_arrive_expect_tx(q_full + st, C::TILE + 1024);
+        mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
 #pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-          tma_load_3d(&tm_q, q_full + st, smem + C::Q_OFF + st * C::TILE + b * C::BLK, b * 64, y,
-                      bh);
-        const size_t vrow = static_cast<size_t>(bh) * Np + y;
-        bulk_load_1d(smem + C::VEC_OFF + st * 1024, lse2 + vrow, 512, q_full + st);
-        bulk_load_1d(smem + C::VEC_OFF + st * 1024 + 512, dvec + vrow, 512, q_full + st);
-        mbar_arrive_expect_tx(do_full + st, C::TILE);
+        for (int b = 0; b < C::NB; ++b) {
+          tma_load_3d(&tm_k, kv_full, smem + C::K_OFF + b * C::BLK, b * 64, j * kT, bh);
+          tma_load_3d(&tm_v, kv_full, smem + C::V_OFF + b * C::BLK, b * 64, j * kT, bh);
+        }
+        kv_issued = w + 1;
+        for (int it = 0; it < n_iter; ++it, ++qr) {
+          const int st = static_cast<int>(qr & 1);
+          const uint32_t u = qr >> 1;
+          if (qr >= 2 && !mbar_wait(qdo_empty + st, (u - 1) & 1, abort, ctl, kSiteBwdProducer)) {
+            ok = false;
+            break;
+          }
+          const int y = (i_start + it) * kT;
+          mbar_arrive_expect_tx(q_full + st, C::TILE + 1024);
 #pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-          tma_load_3d(&tm_do, do_full + st, smem + C::DO_OFF + st * C::TILE + b * C::BLK, b * 64,
-                      y, bh);
-        last[st] = static_cast<int>(u);
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_3d(&tm_q, q_full + st, smem + C::Q_OFF + st * C::TILE + b * C::BLK, b * 64,
+                        y, bh);
+          const size_t vrow = static_cast<size_t>(bh) * Np + y;
+          bulk_load_1d(smem + C::VEC_OFF + st * 1024, lse2 + vrow, 512, q_full + st);
+          bulk_load_1d(smem + C::VEC_OFF + st * 1024 + 512, dvec + vrow, 512, q_full + st);
+          mbar_arrive_expect_tx(do_full + st, C::TILE);
+#pragma unroll
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_3d(&tm_do, do_full + st, smem + C::DO_OFF + st * C::TILE + b * C::BLK,
+                        b * 64, y, bh);
+          last[st] = static_cast<int>(u);
+        }
+        if (!ok) break;
+        if (!producer_request_item(w, nxt_full, nxt_empty, nxt_resp, abort, ctl,
+                                   kSiteBwdProducer, nxt_pending, nxt_pending_par))
+          break;
       }
       if (*abort) {
-        drain_wait(kv_full, 0, ctl);
+        if (kv_issued > 0) drain_wait(kv_full, static_cast<uint32_t>(kv_issued - 1) & 1, ctl);
         for (int s = 0; s < 2; ++s)
           if (last[s] >= 0) {
             drain_wait(q_full + s, last[s] & 1, ctl);
             drain_wait(do_full + s, last[s] & 1, ctl);
           }
+        if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
       }
     }
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
     // All lanes run the schedule; the elected lane issues MMAs and commits.
-    {
-      const bool leader = elect_one();
-      constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S^T, dP^T
-      constexpr uint32_t kIdescAcc = idesc_bf16(kT, D, 0, 1);  // dV, dK (B MN-major)
-      const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);           // K-major (A)
-      const SDesc v_desc = sdesc(sbase + C::V_OFF, 16, 1024);           // K-major (A)
-      const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);           // K-major (B of S^T)
-      const SDesc do_desc = sdesc(sbase + C::DO_OFF, 16, 1024);         // K-major (B of dP^T)
-      const SDesc q_mn = sdesc(sbase + C::Q_OFF, C::BLK, 1024);         // MN-major (B of dK)
-      const SDesc do_mn = sdesc(sbase + C::DO_OFF, C::BLK, 1024);       // MN-major (B of dV)
-      auto issue_s = [&](int it) -> bool {  // S^T = K_j Q_i^T -> region A
-        const int st = it & 1;
-        if (!wait_all(q_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
-          return false;
-        tc_fence_after();
-        if (leader) {
-          const SDesc qd = q_desc + st * C::TILE;
-#pragma unroll
-          for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-            mma_ss(tmem + kKvColS, k_desc + off, qd + off, kIdescSq, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(s_full);
-        }
+    const bool leader = elect_one();
+    constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S^T, dP^T
+    constexpr uint32_t kIdescAcc = idesc_bf16(kT, D, 0, 1);  // dV, dK (B MN-major)
+    const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);           // K-major (A)
+    const SDesc v_desc = sdesc(sbase + C::V_OFF, 16, 1024);           // K-major (A)
+    const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);           // K-major (B of S^T)
+    const SDesc do_desc = sdesc(sbase + C::DO_OFF, 16, 1024);         // K-major (B of dP^T)
+    const SDesc q_mn = sdesc(sbase + C::Q_OFF, C::BLK, 1024);         // MN-major (B of dK)
+    const SDesc do_mn = sdesc(sbase + C::DO_OFF, C::BLK, 1024);       // MN-major (B of dV)
+    uint32_t qbase = 0;  // query tiles of the previous items (ring uses, barrier phases)
+    int n_iter = 0, s_done = 0, dp_done = 0, released = 0;
+    auto release_kv = [&]() {  // after the item's last S^T and dP^T
+      if (!released && s_done == n_iter && dp_done == n_iter) {
+        if (leader) mma_commit(kv_empty);
         __syncwarp();
-        return true;
-      };
-      auto issue_dp = [&](int it) -> bool {  // dP^T = V_j dO_i^T -> region B
-        const int st = it & 1;
-        if (!wait_all(do_full + st, static_cast<uint32_t>(it >> 1) & 1, abort, ctl, kSiteBwdMma))
-          return false;
-        tc_fence_after();
-        if (leader) {
-          const SDesc dd = do_desc + st * C::TILE;
+        released = 1;
+      }
+    };
+    auto issue_s = [&](int it) -> bool {  // S^T = K_j Q_i^T -> region A
+      const uint32_t g = qbase + it;
+      const int st = static_cast<int>(g & 1);
+      if (!wait_all(q_full + st, (g >> 1) & 1, abort, ctl, kSiteBwdMma)) return false;
+      tc_fence_after();
+      if (leader) {
+        const SDesc qd = q_desc + st * C::TILE;
 #pragma unroll
-          for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-            mma_ss(tmem + kKvColDP, v_desc + off, dd + off, kIdescSq, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(dp_full);
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          mma_ss(tmem + kKvColS, k_desc + off, qd + off, kIdescSq, kk > 0 ? 1u : 0u);
         }
-        __syncwarp();
-        return true;
-      };
-      // S^T_{i+1} overwrites P^T_i in A: issued after dV_i (same thread, in
-      // order); the softmax is done with A once it signalled p_full.
-      // dP^T_{i+1} overwrites dS^T_i in B: issued after dK_i, in order.
-      bool ok = wait_all(kv_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
+        mma_commit(s_full);
+      }
+      __syncwarp();
+      ++s_done;
+      release_kv();
+      return true;
+    };
+    auto issue_dp = [&](int it) -> bool {  // dP^T = V_j dO_i^T -> region B
+      const uint32_t g = qbase + it;
+      const int st = static_cast<int>(g & 1);
+      if (!wait_all(do_full + st, (g >> 1) & 1, abort, ctl, kSiteBwdMma)) return false;
+      tc_fence_after();
+      if (leader) {
+        const SDesc dd = do_desc + st * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          mma_ss(tmem + kKvColDP, v_desc + off, dd + off, kIdescSq, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(dp_full);
+      }
+      __syncwarp();
+      ++dp_done;
+      release_kv();
+      return true;
+    };
+    // S^T_{i+1} overwrites P^T_i in A: issued after dV_i (same thread, in
+    // order); the softmax is done with A once it signalled p_full.
+    // dP^T_{i+1} overwrites dS^T_i in B: issued after dK_i, in order.
+    bool ok = true;
+    int idx = 0;
+    for (int w = 0; ok; ++w) {
+      if (!next_item(w, idx, kSiteBwdMma)) break;
+      if (idx < 0) break;
+      int bh, j, i_start;
+      decode(idx, bh, j, i_start, n_iter);
+      s_done = dp_done = released = 0;
+      ok = wait_all(kv_full, static_cast<uint32_t>(w) & 1, abort, ctl, kSiteBwdMma) &&
+           issue_s(0) && issue_dp(0);
       for (int it = 0; ok && it < n_iter; ++it) {
-        const int st = it & 1;
+        const uint32_t g = qbase + it;
+        const int st = static_cast<int>(g & 1);
         const SDesc qm = q_mn + st * C::TILE;
         const SDesc dm = do_mn + st * C::TILE;
         // dV += P^T dO_i: query k-step kk (16 queries) lives in columns
         // 64*(kk/4) + 8*(kk%4) of region A.
-        if (!wait_all(p_full, it & 1, abort, ctl, kSiteBwdMma)) break;
+        if (!wait_all(p_full, g & 1, abort, ctl, kSiteBwdMma)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         if (leader) {
 #pragma unroll
@@ -323,10 +398,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                    (it > 0 || kk > 0) ? 1u : 0u);
         }
         __syncwarp();
-        if (FA_BWD_EARLY_S && it + 1 < n_iter && !issue_s(it + 1)) break;
-        if (!wait_all(ds_full, it & 1, abort, ctl, kSiteBwdMma)) break;
+        if (FA_BWD_EARLY_S && it + 1 < n_iter && !issue_s(it + 1)) {
+          ok = false;
+          break;
+        }
+        if (!wait_all(ds_full, g & 1, abort, ctl, kSiteBwdMma)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        if (!FA_BWD_EARLY_S && it + 1 < n_iter && !issue_s(it + 1)) break;
+        if (!FA_BWD_EARLY_S && it + 1 < n_iter && !issue_s(it + 1)) {
+          ok = false;
+          break;
+        }
         // dK += dS^T Q_i: dS^T k-step kk at column 128 + 64*(kk/4) + 8*(kk%4).
         if (leader) {
 #pragma unroll
@@ -337,9 +421,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(qdo_empty + st);
         }
         __syncwarp();
-        if (it + 1 < n_iter && !issue_dp(it + 1)) break;
+        if (it + 1 < n_iter && !issue_dp(it + 1)) {
+          ok = false;
+          break;
+        }
       }
+      if (!ok) break;
       if (leader) mma_commit(kv_done);
+      __syncwarp();
+      qbase += static_cast<uint32_t>(n_iter);
     }
     __syncwarp();
   } else {
@@ -349,104 +439,118 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t col_s = kKvColS + 64 * h;    // this half's S^T, then P^T
     const uint32_t col_dp = kKvColDP + 64 * h;  // this half's dP^T, then dS^T
-    const int k_idx = j * kT + kr;
-    const bool key_ok = k_idx < N;
+    uint32_t qbase = 0;  // query tiles of the previous items (barrier phases)
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      const int i = i_start + it;
-      const int st = it & 1;
-      // LSE2 and D of this half's 64 queries, staged by the producer with
-      // the Q tile (q_full[st] completed before S^T, hence before s_full).
-      const float* l2 = reinterpret_cast<const float*>(smem + C::VEC_OFF + st * 1024) + 64 * h;
-      const float* dd = l2 + 128;
-      const bool diag = CAUSAL && (i == j);
-      if (!wait_all(s_full, it & 1, abort, ctl, kSiteBwdSoftmax)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sv[2][32];
-      tmem_ld32(lane_base + col_s, sv[0]);
-      tmem_ld32(lane_base + col_s + 32, sv[1]);
-      tmem_wait_ld();
-      const float2 sc2 = make_float2(scale_log2, scale_log2);
-      // queries of this half this key row sees: all, none (key past N), or
-      // q >= key on the diagonal tile
-      const int qlo = !key_ok ? 64 : (diag ? kr - 64 * h : 0);
-      uint32_t pk[32];  // P^T of this half, bf16 pairs
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 lv = *reinterpret_cast<const float4*>(l2 + c * 32 + e);
-          const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e]),
-                                                    __uint_as_float(sv[c][e + 1])),
-                                        sc2, make_float2(-lv.x, -lv.y));
-          const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e + 2]),
-                                                    __uint_as_float(sv[c][e + 3])),
-                                        sc2, make_float2(-lv.z, -lv.w));
-          // one pair in three on the FMA pipe, the rest on the MUFU
-          float2 p01, p23;
-          if (((c * 16 + e / 2) % 3) == 2)
-            p01 = exp2_fma2(x01);
-          else
-            p01 = make_float2(ex2(x01.x), ex2(x01.y));
-          if (((c * 16 + e / 2 + 1) % 3) == 2)
-            p23 = exp2_fma2(x23);
-          else
-            p23 = make_float2(ex2(x23.x), ex2(x23.y));
-          const int q0 = c * 32 + e;  // query within this half
-          if (q0 + 0 < qlo) p01.x = 0.f;
-          if (q0 + 1 < qlo) p01.y = 0.f;
-          if (q0 + 2 < qlo) p23.x = 0.f;
-          if (q0 + 3 < qlo) p23.y = 0.f;
-          pk[c * 16 + e / 2] = pack_bf16(p01.x, p01.y);
-          pk[c * 16 + e / 2 + 1] = pack_bf16(p23.x, p23.y);
+    int idx = 0;
+    for (int w = 0; ok; ++w) {
+      if (!next_item(w, idx, kSiteBwdSoftmax)) break;
+      if (idx < 0) break;
+      int bh, j, i_start, n_iter;
+      decode(idx, bh, j, i_start, n_iter);
+      const int k_idx = j * kT + kr;
+      const bool key_ok = k_idx < N;
+      for (int it = 0; it < n_iter; ++it) {
+        const int i = i_start + it;
+        const uint32_t g = qbase + it;
+        const int st = static_cast<int>(g & 1);
+        // LSE2 and D of this half's 64 queries, staged by the producer with
+        // the Q tile (q_full[st] completed before S^T, hence before s_full).
+        const float* l2 = reinterpret_cast<const float*>(smem + C::VEC_OFF + st * 1024) + 64 * h;
+        const float* dd = l2 + 128;
+        const bool diag = CAUSAL && (i == j);
+        if (!wait_all(s_full, g & 1, abort, ctl, kSiteBwdSoftmax)) {
+          ok = false;
+          break;
         }
-      }
-      // P^T -> columns [col_s, col_s + 32): already read above.
-      tmem_st32(lane_base + col_s, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full);
+        tc_fence_after();
+        uint32_t sv[2][32];
+        tmem_ld32(lane_base + col_s, sv[0]);
+        tmem_ld32(lane_base + col_s + 32, sv[1]);
+        tmem_wait_ld();
+        const float2 sc2 = make_float2(scale_log2, scale_log2);
+        // queries of this half this key row sees: all, none (key past N), or
+        // q >= key on the diagonal tile
+        const int qlo = !key_ok ? 64 : (diag ? kr - 64 * h : 0);
+        uint32_t pk[32];  // P^T of this half, bf16 pairs
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 lv = *reinterpret_cast<const float4*>(l2 + c * 32 + e);
+            const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e]),
+                                                      __uint_as_float(sv[c][e + 1])),
+                                          sc2, make_float2(-lv.x, -lv.y));
+            const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e + 2]),
+                                                      __uint_as_float(sv[c][e + 3])),
+                                          sc2, make_float2(-lv.z, -lv.w));
+            // one pair in FA_BWD_POLY_EVERY on the FMA pipe, the rest on the MUFU
+            float2 p01, p23;
+            if (FA_BWD_POLY_EVERY > 0 && ((c * 16 + e / 2) % kBwdPolyMod) == kBwdPolyMod - 1)
+              p01 = exp2_fma2(x01);
+            else
+              p01 = make_float2(ex2(x01.x), ex2(x01.y));
+            if (FA_BWD_POLY_EVERY > 0 &&
+                ((c * 16 + e / 2 + 1) % kBwdPolyMod) == kBwdPolyMod - 1)
+              p23 = exp2_fma2(x23);
+            else
+              p23 = make_float2(ex2(x23.x), ex2(x23.y));
+            const int q0 = c * 32 + e;  // query within this half
+            if (q0 + 0 < qlo) p01.x = 0.f;
+            if (q0 + 1 < qlo) p01.y = 0.f;
+            if (q0 + 2 < qlo) p23.x = 0.f;
+            if (q0 + 3 < qlo) p23.y = 0.f;
+            pk[c * 16 + e / 2] = pack_bf16(p01.x, p01.y);
+            pk[c * 16 + e / 2 + 1] = pack_bf16(p23.x, p23.y);
+          }
+        }
+        // P^T -> columns [col_s, col_s + 32): already read above.
+        tmem_st32(lane_base + col_s, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
 
-      if (!wait_all(dp_full, it & 1, abort, ctl, kSiteBwdSoftmax)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t dpv[2][32];
-      tmem_ld32(lane_base + col_dp, dpv[0]);
-      tmem_ld32(lane_base + col_dp + 32, dpv[1]);
-      tmem_wait_ld();
-      uint32_t dsk[32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 dv4 = *reinterpret_cast<const float4*>(dd + c * 32 + e);
-          const uint32_t p01 = pk[c * 16 + e / 2], p23 = pk[c * 16 + e / 2 + 1];
-          const float d0 = bf16lo(p01) * (__uint_as_float(dpv[c][e + 0]) - dv4.x);
-          const float d1 = bf16hi(p01) * (__uint_as_float(dpv[c][e + 1]) - dv4.y);
-          const float d2 = bf16lo(p23) * (__uint_as_float(dpv[c][e + 2]) - dv4.z);
-          const float d3 = bf16hi(p23) * (__uint_as_float(dpv[c][e + 3]) - dv4.w);
-          dsk[c * 16 + e / 2] = pack_bf16(d0, d1);
-          dsk[c * 16 + e / 2 + 1] = pack_bf16(d2, d3);
+        if (!wait_all(dp_full, g & 1, abort, ctl, kSiteBwdSoftmax)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        uint32_t dpv[2][32];
+        tmem_ld32(lane_base + col_dp, dpv[0]);
+        tmem_ld32(lane_base + col_dp + 32, dpv[1]);
+        tmem_wait_ld();
+        uint32_t dsk[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 dv4 = *reinterpret_cast<const float4*>(dd + c * 32 + e);
+            const uint32_t p01 = pk[c * 16 + e / 2], p23 = pk[c * 16 + e / 2 + 1];
+            const float d0 = bf16lo(p01) * (__uint_as_float(dpv[c][e + 0]) - dv4.x);
+            const float d1 = bf16hi(p01) * (__uint_as_float(dpv[c][e + 1]) - dv4.y);
+            const float d2 = bf16lo(p23) * (__uint_as_float(dpv[c][e + 2]) - dv4.z);
+            const float d3 = bf16hi(p23) * (__uint_as_float(dpv[c][e + 3]) - dv4.w);
+            dsk[c * 16 + e / 2] = pack_bf16(d0, d1);
+            dsk[c * 16 + e / 2 + 1] = pack_bf16(d2, d3);
+          }
+        }
+        // dS^T -> columns [col_dp, col_dp + 32): dP^T values there were read.
+        tmem_st32(lane_base + col_dp, dsk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(ds_full);
       }
-      // dS^T -> columns [col_dp, col_dp + 32): dP^T values there were read.
-      tmem_st32(lane_base + col_dp, dsk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(ds_full);
-    }
-    // Epilogue: dV (unscaled) and dK (times scale), 16-column steps split
-    // between the two warpgroups.
-    if (ok && wait_all(kv_done, 0, abort, ctl, kSiteBwdEpilogue)) {
+      if (!ok) break;
+      // Epilogue: dV (unscaled) and dK (times scale), 16-column steps split
+      // between the two warpgroups.  kv_done completes once per item; the
+      // next item's first dV/dK MMAs (accumulate off) come after this
+      // warpgroup's next P^T / dS^T, so the loads below are complete by then.
+      if (!wait_all(kv_done, static_cast<uint32_t>(w) & 1, abort, ctl, kSiteBwdEpilogue)) break;
       tc_fence_after();
       const size_t row = (static_cast<size_t>(bh) * N + k_idx) * D;
       store_row_bf16<D>(lane_base + kKvColDV, 1.f, dv + row, key_ok, h);
       store_row_bf16<D>(lane_base + kKvColDK, scale, dk + row, key_ok, h);
+      tc_fence_before();
+      qbase += static_cast<uint32_t>(n_iter);
     }
   }
 
@@ -474,9 +578,10 @@ struct QCfg : Shape<D> {
   static constexpr int K_OFF = DO_OFF + S::TILE;      // [NK]
   static constexpr int V_OFF = K_OFF + NK * S::TILE;  // [NV]
   static constexpr int BAR_OFF = V_OFF + NV * S::TILE;
-  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 5;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int SMEM = MISC_OFF + 16 + 1024;
+  static constexpr int NBAR = 12 + 2 * NK + 2 * NV;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
+  static constexpr int SMEM = MISC_OFF + 48 + 1024;
+  static_assert(MISC_OFF % 16 == 0, "next-item responses need 16-byte alignment");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -499,29 +604,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* q_full = bars + 0;  // Q_i and dO_i
-  uint64_t* dq_done = bars + 1;
-  uint64_t* k_full = bars + 2;          // [NK]
+  uint64_t* q_full = bars + 0;   // Q_i and dO_i
+  uint64_t* q_empty = bars + 1;  // the item's S and dP MMAs are done with Q_i, dO_i
+  uint64_t* dq_done = bars + 2;
+  uint64_t* k_full = bars + 3;          // [NK]
   uint64_t* k_empty = k_full + C::NK;   // [NK]
   uint64_t* v_full = k_empty + C::NK;   // [NV]
   uint64_t* v_empty = v_full + C::NV;   // [NV]
   uint64_t* s_full = v_empty + C::NV;   // [2] per S buffer
-  uint64_t* ds_full = s_full + 2;         // [2] per S buffer
+  uint64_t* ds_full = s_full + 2;       // [2] per S buffer
   uint64_t* dp_full = ds_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  uint64_t* nxt_full = dp_full + 1;     // [2] next-item requests
+  uint64_t* nxt_empty = nxt_full + 2;   // [2]
+  uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 36);
 
   const int warp = warp_id();
   const int lane = lane_id();
   const int n_t = (N + kT - 1) / kT;
   const int Np = n_t * kT;
-  int bh, t;
-  group_major(n_t, BH, group, bh, t);
-  const int i = n_t - 1 - t;  // longest query tiles first when causal
-  const int n_kv = CAUSAL ? i + 1 : n_t;
+  // Query tile i and the key tiles it sees for work item idx (group-major,
+  // longest query tiles first when causal).
+  auto decode = [&](int idx, int& bh, int& i, int& n_kv) {
+    int t;
+    group_major(idx, n_t, BH, group, bh, t);
+    i = n_t - 1 - t;
+    n_kv = CAUSAL ? i + 1 : n_t;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     mbar_init(dq_done, 1);
     for (int s = 0; s < C::NK; ++s) {
       mbar_init(k_full + s, 1);
@@ -534,6 +648,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
       mbar_init(ds_full + b, 2 * kT);
+      mbar_init(nxt_full + b, 1);
+      mbar_init(nxt_empty + b, 9);  // MMA warp + 8 softmax warps
     }
     mbar_init(dp_full, 1);
     *abort = 0;
@@ -547,6 +663,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  auto next_item = [&](int it, int& idx, int site) -> bool {
+    return next_work_item(it, idx, nxt_full, nxt_empty, nxt_resp, abort, ctl, site);
+  };
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -560,117 +679,188 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < C::NK; ++s) last_k[s] = -1;
 #pragma unroll
       for (int s = 0; s < C::NV; ++s) last_v[s] = -1;
-      mbar_arrive_expect_tx(q_full, 2 * C::TILE);
-#pragma unroll
-      for (int b = 0; b < C::NB; ++b) {
-        tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + b * C::BLK, b * 64, i * kT, bh);
-        tma_load_3d(&tm_do, q_full, smem + C::DO_OFF + b * C::BLK, b * 64, i * kT, bh);
-      }
-      for (int jj = 0; jj < n_kv; ++jj) {
-        const int sk = jj % C::NK, sv = jj % C::NV;
-        const uint32_t uk = static_cast<uint32_t>(jj / C::NK);
-        const uint32_t uv = static_cast<uint32_t>(jj / C::NV);
-        if (jj >= C::NK && !mbar_wait(k_empty + sk, (uk - 1) & 1, abort, ctl, kSiteBwdProducer))
+      int q_issued = 0;
+      int nxt_pending = -1;
+      uint32_t nxt_pending_par = 0;
+      uint32_t kr = 0;  // key tiles streamed so far (ring uses of both rings)
+      int idx = static_cast<int>(blockIdx.x);
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        if (it > 0) {
+          if (!producer_take_item(it, idx, nxt_full, nxt_resp, abort, ctl, kSiteBwdProducer))
+            break;
+          nxt_pending = -1;
+          if (idx < 0) break;
+        }
+        int bh, i, n_kv;
+        decode(idx, bh, i, n_kv);
+        if (it > 0 &&
+            !mbar_wait(q_empty, static_cast<uint32_t>(it - 1) & 1, abort, ctl, kSiteBwdProducer))
           break;
-        mbar_arrive_expect_tx(k_full + sk, C::TILE);
+        mbar_arrive_expect_tx(q_full, 2 * C::TILE);
 #pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-          tma_load_3d(&tm_k, k_full + sk, smem + C::K_OFF + sk * C::TILE + b * C::BLK, b * 64,
-                      jj * kT, bh);
-        last_k[sk] = static_cast<int>(uk);
-        if (jj >= C::NV && !mbar_wait(v_empty + sv, (uv - 1) & 1, abort, ctl, kSiteBwdProducer))
+        for (int b = 0; b < C::NB; ++b) {
+          tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + b * C::BLK, b * 64, i * kT, bh);
+          tma_load_3d(&tm_do, q_full, smem + C::DO_OFF + b * C::BLK, b * 64, i * kT, bh);
+        }
+        q_issued = it + 1;
+        for (int jj = 0; jj < n_kv; ++jj, ++kr) {
+          const int sk = static_cast<int>(kr % C::NK), sv = static_cast<int>(kr % C::NV);
+          const uint32_t uk = kr / C::NK, uv = kr / C::NV;
+          if (kr >= C::NK &&
+              !mbar_wait(k_empty + sk, (uk - 1) & 1, abort, ctl, kSiteBwdProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(k_full + sk, C::TILE);
+#pragma unroll
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_3d(&tm_k, k_full + sk, smem + C::K_OFF + sk * C::TILE + b * C::BLK, b * 64,
+                        jj * kT, bh);
+          last_k[sk] = static_cast<int>(uk);
+          if (kr >= C::NV &&
+              !mbar_wait(v_empty + sv, (uv - 1) & 1, abort, ctl, kSiteBwdProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(v_full + sv, C::TILE);
+#pragma unroll
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_3d(&tm_v, v_full + sv, smem + C::V_OFF + sv * C::TILE + b * C::BLK, b * 64,
+                        jj * kT, bh);
+          last_v[sv] = static_cast<int>(uv);
+        }
+        if (!ok) break;
+        if (!producer_request_item(it, nxt_full, nxt_empty, nxt_resp, abort, ctl,
+                                   kSiteBwdProducer, nxt_pending, nxt_pending_par))
           break;
-        mbar_arrive_expect_tx(v_full + sv, C::TILE);
-#pragma unroll
-        for (int b = 0; b < C::NB; ++b)
-          tma_load_3d(&tm_v, v_full + sv, smem + C::V_OFF + sv * C::TILE + b * C::BLK, b * 64,
-                      jj * kT, bh);
-        last_v[sv] = static_cast<int>(uv);
       }
       if (*abort) {
-        drain_wait(q_full, 0, ctl);
+        if (q_issued > 0) drain_wait(q_full, static_cast<uint32_t>(q_issued - 1) & 1, ctl);
         for (int s = 0; s < C::NK; ++s)
           if (last_k[s] >= 0) drain_wait(k_full + s, last_k[s] & 1, ctl);
         for (int s = 0; s < C::NV; ++s)
           if (last_v[s] >= 0) drain_wait(v_full + s, last_v[s] & 1, ctl);
+        if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
       }
     }
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
     // All lanes run the schedule; the elected lane issues MMAs and commits.
-    {
-      const bool leader = elect_one();
-      constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S, dP
-      constexpr uint32_t kIdescDq = idesc_bf16(kT, D, 0, 1);   // dQ (B = K_j MN-major)
-      const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);     // K-major (A of S)
-      const SDesc do_desc = sdesc(sbase + C::DO_OFF, 16, 1024);   // K-major (A of dP)
-      const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);     // K-major (B of S)
-      const SDesc v_desc = sdesc(sbase + C::V_OFF, 16, 1024);     // K-major (B of dP)
-      const SDesc k_mn = sdesc(sbase + C::K_OFF, C::BLK, 1024);   // MN-major (B of dQ)
-      auto issue_s = [&](int jj) -> bool {  // S_jj = Q K_jj^T -> buffer jj % 2
-        const int s = jj % C::NK;
-        if (!wait_all(k_full + s, (jj / C::NK) & 1, abort, ctl, kSiteBwdMma)) return false;
-        tc_fence_after();
-        if (leader) {
-          const SDesc kd = k_desc + s * C::TILE;
-#pragma unroll
-          for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-            mma_ss(tmem + kQColS + (jj & 1) * kT, q_desc + off, kd + off, kIdescSq,
-                   kk > 0 ? 1u : 0u);
-          }
-          mma_commit(s_full + (jj & 1));
-        }
+    const bool leader = elect_one();
+    constexpr uint32_t kIdescSq = idesc_bf16(kT, kT, 0, 0);  // S, dP
+    constexpr uint32_t kIdescDq = idesc_bf16(kT, D, 0, 1);   // dQ (B = K_j MN-major)
+    const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);     // K-major (A of S)
+    const SDesc do_desc = sdesc(sbase + C::DO_OFF, 16, 1024);   // K-major (A of dP)
+    const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);     // K-major (B of S)
+    const SDesc v_desc = sdesc(sbase + C::V_OFF, 16, 1024);     // K-major (B of dP)
+    const SDesc k_mn = sdesc(sbase + C::K_OFF, C::BLK, 1024);   // MN-major (B of dQ)
+    // Running counts across items: key tiles (ring uses) before this item,
+    // which also number the S buffers (buffer g & 1 for the g-th S).
+    uint32_t kbase = 0;
+    int n_kv = 0, released = 0, s_done = 0, dp_done = 0;
+    auto release_q = [&]() {  // after the item's last S and dP
+      if (!released && s_done == n_kv && dp_done == n_kv) {
+        if (leader) mma_commit(q_empty);
         __syncwarp();
-        return true;
-      };
-      auto issue_dp = [&](int jj) -> bool {  // dP_jj = dO V_jj^T, then V_jj is free
-        const int s = jj % C::NV;
-        if (!wait_all(v_full + s, (jj / C::NV) & 1, abort, ctl, kSiteBwdMma)) return false;
-        tc_fence_after();
-        if (leader) {
-          const SDesc vd = v_desc + s * C::TILE;
+        released = 1;
+      }
+    };
+    auto issue_s = [&](int jj) -> bool {  // S_jj = Q K_jj^T -> buffer g % 2
+      const uint32_t g = kbase + jj;
+      const int s = static_cast<int>(g % C::NK);
+      if (!wait_all(k_full + s, (g / C::NK) & 1, abort, ctl, kSiteBwdMma)) return false;
+      tc_fence_after();
+      if (leader) {
+        const SDesc kd = k_desc + s * C::TILE;
 #pragma unroll
-          for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-            mma_ss(tmem + kQColDP, do_desc + off, vd + off, kIdescSq, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(dp_full);
-          mma_commit(v_empty + s);
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          mma_ss(tmem + kQColS + (g & 1) * kT, q_desc + off, kd + off, kIdescSq,
+                 kk > 0 ? 1u : 0u);
         }
-        __syncwarp();
-        return true;
-      };
-      // Order: S_0, dP_0, S_1, [dS_0] dP_1, dQ_0, S_2, [dS_1] dP_2, dQ_1, ...
-      // so the tensor core computes S_{j+1} while the softmax warps form dS_j,
-      // and dP_{j+1} is ready soon after.  S_{j+2} reuses S_j's buffer after
-      // dQ_j has read dS_j (same thread, in order) and the softmax released it
-      // (ds_full waited); dP_{j+1} overwrites dP_j once ds_full(j) says the
-      // softmax has read it.
-      bool ok = wait_all(q_full, 0, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
+        mma_commit(s_full + (g & 1));
+      }
+      __syncwarp();
+      ++s_done;
+      release_q();
+      return true;
+    };
+    auto issue_dp = [&](int jj) -> bool {  // dP_jj = dO V_jj^T, then V_jj is free
+      const uint32_t g = kbase + jj;
+      const int s = static_cast<int>(g % C::NV);
+      if (!wait_all(v_full + s, (g / C::NV) & 1, abort, ctl, kSiteBwdMma)) return false;
+      tc_fence_after();
+      if (leader) {
+        const SDesc vd = v_desc + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          mma_ss(tmem + kQColDP, do_desc + off, vd + off, kIdescSq, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(dp_full);
+        mma_commit(v_empty + s);
+      }
+      __syncwarp();
+      ++dp_done;
+      release_q();
+      return true;
+    };
+    // Order: S_0, dP_0, S_1, [dS_0] dP_1, dQ_0, S_2, [dS_1] dP_2, dQ_1, ...
+    // so the tensor core computes S_{j+1} while the softmax warps form dS_j,
+    // and dP_{j+1} is ready soon after.  S_{j+2} reuses S_j's buffer after
+    // dQ_j has read dS_j (same thread, in order) and the softmax released it
+    // (ds_full waited); dP_{j+1} overwrites dP_j once ds_full(j) says the
+    // softmax has read it.
+    bool ok = true;
+    int idx = 0;
+    for (int it = 0; ok; ++it) {
+      if (!next_item(it, idx, kSiteBwdMma)) break;
+      if (idx < 0) break;
+      int bh, i;
+      decode(idx, bh, i, n_kv);
+      released = s_done = dp_done = 0;
+      ok = wait_all(q_full, static_cast<uint32_t>(it) & 1, abort, ctl, kSiteBwdMma) &&
+           issue_s(0) && issue_dp(0);
       if (ok && n_kv > 1) ok = issue_s(1);
       for (int jj = 0; ok && jj < n_kv; ++jj) {
-        const int s = jj % C::NK;
-        if (!wait_all(ds_full + (jj & 1), (jj >> 1) & 1, abort, ctl, kSiteBwdMma)) break;
+        const uint32_t g = kbase + jj;
+        const int s = static_cast<int>(g % C::NK);
+        if (!wait_all(ds_full + (g & 1), (g >> 1) & 1, abort, ctl, kSiteBwdMma)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        if (FA_BWD_EARLY_DP && jj + 1 < n_kv && !issue_dp(jj + 1)) break;
+        if (FA_BWD_EARLY_DP && jj + 1 < n_kv && !issue_dp(jj + 1)) {
+          ok = false;
+          break;
+        }
         // dQ += dS_jj K_jj: key k-step kk (16 keys) of dS at column
         // 64*(kk/4) + 8*(kk%4) of the S buffer.
         if (leader) {
           const SDesc km = k_mn + s * C::TILE;
 #pragma unroll
           for (int kk = 0; kk < kT / 16; ++kk)
-            mma_ts(tmem + kQColDQ, tmem + kQColS + (jj & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
+            mma_ts(tmem + kQColDQ, tmem + kQColS + (g & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
                    km + kk * 2048, kIdescDq,
                    (jj > 0 || kk > 0) ? 1u : 0u);
           mma_commit(k_empty + s);
         }
         __syncwarp();
-        if (!FA_BWD_EARLY_DP && jj + 1 < n_kv && !issue_dp(jj + 1)) break;
-        if (jj + 2 < n_kv && !issue_s(jj + 2)) break;
+        if (!FA_BWD_EARLY_DP && jj + 1 < n_kv && !issue_dp(jj + 1)) {
+          ok = false;
+          break;
+        }
+        if (jj + 2 < n_kv && !issue_s(jj + 2)) {
+          ok = false;
+          break;
+        }
       }
+      if (!ok) break;
       if (leader) mma_commit(dq_done);
+      __syncwarp();
+      kbase += static_cast<uint32_t>(n_kv);
     }
     __syncwarp();
   } else {
@@ -678,57 +868,71 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2;
     const int qr = threadIdx.x & 127;  // query row == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int q_idx = i * kT + qr;
-    const float my_l2 = lse2[static_cast<size_t>(bh) * Np + q_idx];  // +inf past N
-    const float my_d = dvec[static_cast<size_t>(bh) * Np + q_idx];
+    uint32_t kbase = 0;  // key tiles of the previous items (S buffer numbering)
     bool ok = true;
-    for (int jj = 0; jj < n_kv; ++jj) {
-      const uint32_t col_s = kQColS + (jj & 1) * kT + 64 * h;
-      if (!wait_all(s_full + (jj & 1), (jj >> 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sv[2][32];
-      tmem_ld32(lane_base + col_s, sv[0]);
-      tmem_ld32(lane_base + col_s + 32, sv[1]);
-      tmem_wait_ld();
-      const int k0 = jj * kT + 64 * h;  // first key of this half
-      // keys k visible to this query: k <= q_idx (causal) and k < N
-      const int lim = min(N, CAUSAL ? q_idx + 1 : N) - k0;
-      float p[64];
+    int idx = 0;
+    for (int it = 0; ok; ++it) {
+      if (!next_item(it, idx, kSiteBwdSoftmax)) break;
+      if (idx < 0) break;
+      int bh, i, n_kv;
+      decode(idx, bh, i, n_kv);
+      const int q_idx = i * kT + qr;
+      const float my_l2 = lse2[static_cast<size_t>(bh) * Np + q_idx];  // +inf past N
+      const float my_d = dvec[static_cast<size_t>(bh) * Np + q_idx];
+      for (int jj = 0; jj < n_kv; ++jj) {
+        const uint32_t g = kbase + jj;
+        const uint32_t col_s = kQColS + (g & 1) * kT + 64 * h;
+        if (!wait_all(s_full + (g & 1), (g >> 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[2][32];
+        tmem_ld32(lane_base + col_s, sv[0]);
+        tmem_ld32(lane_base + col_s + 32, sv[1]);
+        tmem_wait_ld();
+        const int k0 = jj * kT + 64 * h;  // first key of this half
+        // keys k visible to this query: k <= q_idx (causal) and k < N
+        const int lim = min(N, CAUSAL ? q_idx + 1 : N) - k0;
+        float p[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float x = fmaf(__uint_as_float(sv[c >> 5][c & 31]), scale_log2, -my_l2);
-        p[c] = (c < lim) ? ex2(x) : 0.f;
-      }
-      if (!wait_all(dp_full, jj & 1, abort, ctl, kSiteBwdSoftmax)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t dpv[2][32];
-      tmem_ld32(lane_base + kQColDP + 64 * h, dpv[0]);
-      tmem_ld32(lane_base + kQColDP + 64 * h + 32, dpv[1]);
-      tmem_wait_ld();
-      uint32_t dsk[32];
+        for (int c = 0; c < 64; ++c) {
+          const float x = fmaf(__uint_as_float(sv[c >> 5][c & 31]), scale_log2, -my_l2);
+          p[c] = (c < lim) ? ex2(x) : 0.f;
+        }
+        if (!wait_all(dp_full, g & 1, abort, ctl, kSiteBwdSoftmax)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t dpv[2][32];
+        tmem_ld32(lane_base + kQColDP + 64 * h, dpv[0]);
+        tmem_ld32(lane_base + kQColDP + 64 * h + 32, dpv[1]);
+        tmem_wait_ld();
+        uint32_t dsk[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int c0 = 2 * c, c1 = 2 * c + 1;
-        const float d0 = p[c0] * (__uint_as_float(dpv[c0 >> 5][c0 & 31]) - my_d);
-        const float d1 = p[c1] * (__uint_as_float(dpv[c1 >> 5][c1 & 31]) - my_d);
-        dsk[c] = pack_bf16(d0, d1);
+        for (int c = 0; c < 32; ++c) {
+          const int c0 = 2 * c, c1 = 2 * c + 1;
+          const float d0 = p[c0] * (__uint_as_float(dpv[c0 >> 5][c0 & 31]) - my_d);
+          const float d1 = p[c1] * (__uint_as_float(dpv[c1 >> 5][c1 & 31]) - my_d);
+          dsk[c] = pack_bf16(d0, d1);
+        }
+        // dS -> columns [col_s, col_s + 32) of the S buffer (already read).
+        tmem_st32(lane_base + col_s, dsk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(ds_full + (g & 1));
       }
-      // dS -> columns [col_s, col_s + 32) of the S buffer (already read).
-      tmem_st32(lane_base + col_s, dsk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(ds_full + (jj & 1));
-    }
-    if (ok && wait_all(dq_done, 0, abort, ctl, kSiteBwdEpilogue)) {
+      if (!ok) break;
+      // dq_done completes once per item; the next item's first dQ MMA
+      // (accumulate off) comes after this warpgroup's next dS, so the loads
+      // below are complete by then.
+      if (!wait_all(dq_done, static_cast<uint32_t>(it) & 1, abort, ctl, kSiteBwdEpilogue)) break;
       tc_fence_after();
       store_row_bf16<D>(lane_base + kQColDQ, scale, dq + (static_cast<size_t>(bh) * N + q_idx) * D,
                         q_idx < N, h);
+      tc_fence_before();
+      kbase += static_cast<uint32_t>(n_kv);
     }
   }
 

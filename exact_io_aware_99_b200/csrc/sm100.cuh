@@ -135,6 +135,58 @@ __device__ __forceinline__ int clc_result_x(const void* resp16) {
   return canceled ? static_cast<int>(x) : -1;
 }
 
+// Work items of a persistent CTA (see clc_try_cancel).  Item 0 is the CTA's
+// own blockIdx.x; item it >= 1 is the answer to the request the producer
+// thread issued while it worked on item it - 1, kept in slot it & 1 of a
+// two-slot ring (16-byte responses `resp`, barriers full[2] / empty[2]); the
+// consumer warps release a slot through `empty` after reading it.
+
+// Consumer side, called by all lanes of a warp.  Returns false when the
+// wait gave up; idx < 0 means the grid has no work left.
+__device__ __forceinline__ bool next_work_item(int it, int& idx, uint64_t* full, uint64_t* empty,
+                                               const uint8_t* resp, volatile int* abort,
+                                               const WaitCtl& ctl, int site) {
+  if (it == 0) {
+    idx = static_cast<int>(blockIdx.x);
+    return true;
+  }
+  const int sl = it & 1;
+  const bool w = mbar_wait(full + sl, static_cast<uint32_t>((it - 1) >> 1) & 1, abort, ctl, site);
+  if (!__all_sync(0xffffffffu, w)) return false;
+  idx = clc_result_x(resp + 16 * sl);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(empty + sl);
+  return true;
+}
+
+// Producer side (one thread): the answer for item it >= 1.
+__device__ __forceinline__ bool producer_take_item(int it, int& idx, uint64_t* full,
+                                                   const uint8_t* resp, volatile int* abort,
+                                                   const WaitCtl& ctl, int site) {
+  const int sl = it & 1;
+  if (!mbar_wait(full + sl, static_cast<uint32_t>((it - 1) >> 1) & 1, abort, ctl, site))
+    return false;
+  idx = clc_result_x(resp + 16 * sl);
+  return true;
+}
+
+// Producer side (one thread): request item it + 1 into slot (it + 1) & 1
+// once the consumers have read that slot's previous answer.  `pending` and
+// `pending_par` record the request in flight (drained on abort).
+__device__ __forceinline__ bool producer_request_item(int it, uint64_t* full, uint64_t* empty,
+                                                      uint8_t* resp, volatile int* abort,
+                                                      const WaitCtl& ctl, int site, int& pending,
+                                                      uint32_t& pending_par) {
+  const int sl = (it + 1) & 1;
+  const uint32_t u = static_cast<uint32_t>(it >> 1);
+  if (u > 0 && !mbar_wait(empty + sl, (u - 1) & 1, abort, ctl, site)) return false;
+  mbar_arrive_expect_tx(full + sl, 16);
+  clc_try_cancel(resp + 16 * sl, full + sl);
+  pending = sl;
+  pending_par = u & 1;
+  return true;
+}
+
 // Contiguous (untiled) bulk copy global -> shared, completion as transaction
 // bytes on `bar`.  Both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
