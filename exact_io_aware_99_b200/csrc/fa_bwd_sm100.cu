@@ -946,13 +946,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ launch
 
-// Heads per group, from the bytes every CTA of a head re-reads (Q and dO for
+// Heads per group, from the bytes every item of a head re-reads (Q and dO for
 // the dK/dV kernel, K and V for the dQ kernel: 4 N d each): a group's share
-// stays within ~64 MB of the 126 MB L2, and the groups are large enough that
-// the longest-first order ends on short CTAs (small groups start their last
-// group's long CTAs at the end and leave SMs idle).
-inline int heads_per_group(long long per_head_bytes, int BH) {
-  int g = static_cast<int>((64LL << 20) / (per_head_bytes > 0 ? per_head_bytes : 1));
+// stays within the L2 share (64 MB causal, 32 MB otherwise); causal groups
+// are large so that the longest-first order ends on short items (small
+// groups start their last group's long items at the end and leave SMs idle).
+inline int heads_per_group(long long per_head_bytes, int BH, bool causal) {
+  int g = static_cast<int>(l2_group_bytes(causal) / (per_head_bytes > 0 ? per_head_bytes : 1));
   return g < 1 ? 1 : (g > BH ? BH : g);
 }
 
@@ -976,7 +976,7 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   // Heads per group: a group's Q, K, V, dO (bf16, 8 N d bytes per head)
   // within ~48 MB of the 126 MB L2.
-  const int group = heads_per_group(4LL * N * D, BH);
+  const int group = heads_per_group(4LL * N * D, BH, CAUSAL);
   const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};
   bwd_dkdv_kernel<D, CAUSAL>

@@ -571,14 +571,15 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   }
   const int n_t = (N + kBM - 1) / kBM;
   const int n_pair = (n_t + 1) / 2;
-  // Heads per group: the operands every CTA of a head re-reads are K and V
-  // (4 N d bytes per head); a group's K and V stay within ~64 MB of the
-  // 126 MB L2 while Q and O stream through.  Large groups also keep the
-  // longest-first order global enough that the last CTAs are short ones
-  // (with 12-head groups the final group's long CTAs started last and left
-  // ~13% of the SMs idle at the end of a causal N = 4096 launch).
+  // Heads per group: the operands every item of a head re-reads are K and V
+  // (4 N d bytes per head); a group's K and V stay within the L2 share
+  // (64 MB causal, 32 MB otherwise) while Q and O stream through.  Causal
+  // launches need the large groups to keep the longest-first order global
+  // enough that the last items are short ones (with 12-head groups the final
+  // group's long items started last and left ~13% of the SMs idle at the end
+  // of a causal N = 4096 launch).
   const long long per_head = 4LL * N * D;
-  int group = static_cast<int>((64LL << 20) / (per_head > 0 ? per_head : 1));
+  int group = static_cast<int>(l2_group_bytes(CAUSAL) / (per_head > 0 ? per_head : 1));
   group = group < 1 ? 1 : (group > BH ? BH : group);
   const long long blocks = static_cast<long long>(BH) * n_pair;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;

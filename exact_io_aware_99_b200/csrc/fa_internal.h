@@ -36,6 +36,21 @@ constexpr int kTileRows = 128;
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
+// L2 share (MB) for the operands a group of heads keeps re-reading; it sets
+// how many heads the kernels work on at a time (group-major work order).
+// Causal launches take larger groups: their work items differ in length and
+// a longest-first order only balances the SMs when it spans many heads.
+// Non-causal items are all equal, so smaller groups (fewer L2 misses) win.
+#ifndef FA_L2_GROUP_MB
+#define FA_L2_GROUP_MB 64
+#endif
+#ifndef FA_L2_GROUP_MB_NONCAUSAL
+#define FA_L2_GROUP_MB_NONCAUSAL 32
+#endif
+inline long long l2_group_bytes(int causal) {
+  return static_cast<long long>(causal ? FA_L2_GROUP_MB : FA_L2_GROUP_MB_NONCAUSAL) << 20;
+}
+
 // --- bf16 tensor-core path (fa_fwd_sm100.cu, fa_bwd_sm100.cu) -------------
 // Tensor maps describe a [BH, N, d] bf16 tensor as 3-D {d, N, BH} with a
 // {64, 128, 1} box and 128-byte swizzle.
