@@ -128,8 +128,9 @@ class ClockSampler:
 
 KERNEL_SOURCES = {
     "bwd": ["exact_io_aware_99_b200/csrc/fa_bwd_sm100.cu", "exact_io_aware_99_b200/csrc/fa_simt.cu",
-            "exact_io_aware_99_b200/csrc/sm100.cuh"],
-    "fwd": ["exact_io_aware_99_b200/csrc/fa_fwd_sm100.cu", "exact_io_aware_99_b200/csrc/sm100.cuh"],
+            "exact_io_aware_99_b200/csrc/sm100.cuh", "exact_io_aware_99_b200/csrc/fa_internal.h"],
+    "fwd": ["exact_io_aware_99_b200/csrc/fa_fwd_sm100.cu", "exact_io_aware_99_b200/csrc/sm100.cuh",
+            "exact_io_aware_99_b200/csrc/fa_internal.h"],
 }
 
 
