@@ -64,7 +64,7 @@ constexpr int kT = 128;  // rows of every tile (keys or queries)
 #endif
 // dK/dV kernel: one column pair in this many takes the FMA-pipe exp2 (0: none).
 #ifndef FA_BWD_POLY_EVERY
-#define FA_BWD_POLY_EVERY 6
+#define FA_BWD_POLY_EVERY 0
 #endif
 constexpr int kBwdPolyMod = FA_BWD_POLY_EVERY > 0 ? FA_BWD_POLY_EVERY : 1;
 constexpr int kThreads = 320;
@@ -129,6 +129,70 @@ __device__ __forceinline__ void store_row_bf16(uint32_t taddr, float mul, __nv_b
       uint4* dst = reinterpret_cast<uint4*>(row + c * 16);
       dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+  }
+}
+
+// P^T of one key row (64 queries of a half tile): 2^(S^T c - LSE2[q]) from
+// the S^T values `sv` and the staged LSE2 vector `l2`, packed to bf16 pairs.
+// MASK zeroes queries q < qlo (diagonal tile, key past N); the unmasked
+// instantiation, used by every tile a whole warp sees unmasked, has no
+// selects in the loop.
+template <bool MASK>
+__device__ __forceinline__ void kv_p_row(const uint32_t (&sv)[2][32], const float* l2, float2 sc2,
+                                         int qlo, uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      const float4 lv = *reinterpret_cast<const float4*>(l2 + c * 32 + e);
+      const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e]),
+                                                __uint_as_float(sv[c][e + 1])),
+                                    sc2, make_float2(-lv.x, -lv.y));
+      const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e + 2]),
+                                                __uint_as_float(sv[c][e + 3])),
+                                    sc2, make_float2(-lv.z, -lv.w));
+      // one pair in FA_BWD_POLY_EVERY on the FMA pipe, the rest on the MUFU
+      float2 p01, p23;
+      if (FA_BWD_POLY_EVERY > 0 && ((c * 16 + e / 2) % kBwdPolyMod) == kBwdPolyMod - 1)
+        p01 = exp2_fma2(x01);
+      else
+        p01 = make_float2(ex2(x01.x), ex2(x01.y));
+      if (FA_BWD_POLY_EVERY > 0 && ((c * 16 + e / 2 + 1) % kBwdPolyMod) == kBwdPolyMod - 1)
+        p23 = exp2_fma2(x23);
+      else
+        p23 = make_float2(ex2(x23.x), ex2(x23.y));
+      if (MASK) {
+        const int q0 = c * 32 + e;  // query within this half
+        if (q0 + 0 < qlo) p01.x = 0.f;
+        if (q0 + 1 < qlo) p01.y = 0.f;
+        if (q0 + 2 < qlo) p23.x = 0.f;
+        if (q0 + 3 < qlo) p23.y = 0.f;
+      }
+      pk[c * 16 + e / 2] = pack_bf16(p01.x, p01.y);
+      pk[c * 16 + e / 2 + 1] = pack_bf16(p23.x, p23.y);
+    }
+  }
+}
+
+// P of one query row (64 keys of a half tile) in the dQ kernel:
+// 2^(S c - LSE2) for keys c < lim, 0 past it (MASK); unmasked rows take the
+// select-free instantiation.
+template <bool MASK>
+__device__ __forceinline__ void dq_p_row(const uint32_t (&sv)[2][32], float scale_log2,
+                                         float my_l2, int lim, float (&p)[64]) {
+  const float2 sc2 = make_float2(scale_log2, scale_log2);
+  const float2 nl2 = make_float2(-my_l2, -my_l2);
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[c >> 5][c & 31]),
+                                            __uint_as_float(sv[c >> 5][(c & 31) + 1])),
+                                sc2, nl2);
+    p[c] = ex2(x.x);
+    p[c + 1] = ex2(x.y);
+    if (MASK) {
+      if (c >= lim) p[c] = 0.f;
+      if (c + 1 >= lim) p[c + 1] = 0.f;
     }
   }
 }
@@ -472,37 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // q >= key on the diagonal tile
         const int qlo = !key_ok ? 64 : (diag ? kr - 64 * h : 0);
         uint32_t pk[32];  // P^T of this half, bf16 pairs
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 lv = *reinterpret_cast<const float4*>(l2 + c * 32 + e);
-            const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e]),
-                                                      __uint_as_float(sv[c][e + 1])),
-                                          sc2, make_float2(-lv.x, -lv.y));
-            const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[c][e + 2]),
-                                                      __uint_as_float(sv[c][e + 3])),
-                                          sc2, make_float2(-lv.z, -lv.w));
-            // one pair in FA_BWD_POLY_EVERY on the FMA pipe, the rest on the MUFU
-            float2 p01, p23;
-            if (FA_BWD_POLY_EVERY > 0 && ((c * 16 + e / 2) % kBwdPolyMod) == kBwdPolyMod - 1)
-              p01 = exp2_fma2(x01);
-            else
-              p01 = make_float2(ex2(x01.x), ex2(x01.y));
-            if (FA_BWD_POLY_EVERY > 0 &&
-                ((c * 16 + e / 2 + 1) % kBwdPolyMod) == kBwdPolyMod - 1)
-              p23 = exp2_fma2(x23);
-            else
-              p23 = make_float2(ex2(x23.x), ex2(x23.y));
-            const int q0 = c * 32 + e;  // query within this half
-            if (q0 + 0 < qlo) p01.x = 0.f;
-            if (q0 + 1 < qlo) p01.y = 0.f;
-            if (q0 + 2 < qlo) p23.x = 0.f;
-            if (q0 + 3 < qlo) p23.y = 0.f;
-            pk[c * 16 + e / 2] = pack_bf16(p01.x, p01.y);
-            pk[c * 16 + e / 2 + 1] = pack_bf16(p23.x, p23.y);
-          }
-        }
+        if (__any_sync(0xffffffffu, qlo > 0))
+          kv_p_row<true>(sv, l2, sc2, qlo, pk);
+        else
+          kv_p_row<false>(sv, l2, sc2, qlo, pk);
         // P^T -> columns [col_s, col_s + 32): already read above.
         tmem_st32(lane_base + col_s, pk);
         tmem_wait_st();
@@ -895,11 +932,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // keys k visible to this query: k <= q_idx (causal) and k < N
         const int lim = min(N, CAUSAL ? q_idx + 1 : N) - k0;
         float p[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float x = fmaf(__uint_as_float(sv[c >> 5][c & 31]), scale_log2, -my_l2);
-          p[c] = (c < lim) ? ex2(x) : 0.f;
-        }
+        if (__any_sync(0xffffffffu, lim < 64))
+          dq_p_row<true>(sv, scale_log2, my_l2, lim, p);
+        else
+          dq_p_row<false>(sv, scale_log2, my_l2, lim, p);
         if (!wait_all(dp_full, g & 1, abort, ctl, kSiteBwdSoftmax)) {
           ok = false;
           break;
