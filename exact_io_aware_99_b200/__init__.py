@@ -6,14 +6,15 @@ used for device memory and streams.
 
 Low-level entry points (same names as the C ABI): ``fa_forward``,
 ``fa_forward_ex``, ``fa_backward``, ``fa_backward_ex``,
-``fa_backward_noalloc``, ``fa_backward_workspace_size``,
+``fa_backward_noalloc``, ``fa_forward_blocksparse``, ``fa_backward_blocksparse``,
+``fa_backward_workspace_size``,
 ``fa_status_string``, ``fa_device_status``, ``fa_set_wait_timeout_ns``,
 ``fa_selftest_wait_timeout``.
 
 Convenience wrappers that allocate outputs with torch:
-``attention_forward(q, k, v, scale=None, causal=False) -> (o, lse)`` and
-``attention_backward(q, k, v, o, do, lse, scale=None, causal=False)
--> (dq, dk, dv)``.
+``attention_forward(q, k, v, scale=None, causal=False, block_mask=None)
+-> (o, lse)`` and ``attention_backward(q, k, v, o, do, lse, scale=None,
+causal=False, block_mask=None) -> (dq, dk, dv)``.
 
 The shared library is loaded on first use of any of these names (so the
 ``build`` submodule can run before it exists); using them without the built
@@ -25,7 +26,8 @@ _NATIVE = {
     "FA_NOALLOC_SCRATCH_BYTES", "FaError", "LIB_PATH", "library", "fa_forward",
     "fa_forward_ex", "fa_backward", "fa_backward_ex", "fa_backward_noalloc",
     "fa_backward_workspace_size", "fa_status_string", "fa_device_status",
-    "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout",
+    "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_forward_blocksparse",
+    "fa_backward_blocksparse",
 }
 _API = {"attention_forward", "attention_backward"}
 

@@ -30,6 +30,7 @@ EXPORTS = (
     "fa_forward", "fa_forward_ex", "fa_backward_workspace_size", "fa_backward",
     "fa_backward_ex", "fa_status_string", "fa_last_cuda_error", "fa_device_status",
     "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_backward_noalloc",
+    "fa_forward_blocksparse", "fa_backward_blocksparse",
 )
 
 # Size of the library's built-in scratch array used by fa_backward_noalloc.
@@ -72,6 +73,11 @@ def _load() -> ctypes.CDLL:
     lib.fa_selftest_wait_timeout.argtypes = [P]
     lib.fa_selftest_wait_timeout.restype = I
     lib.fa_backward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P]
+    lib.fa_forward_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, F, I, P, I, P]
+    lib.fa_forward_blocksparse.restype = I
+    lib.fa_backward_blocksparse.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I,
+                                            P, S, P]
+    lib.fa_backward_blocksparse.restype = I
     lib.fa_backward_noalloc.restype = I
     return lib
 
@@ -172,3 +178,23 @@ def fa_backward_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, caus
                                   _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
                                   int(bool(causal)), _stream(stream))
     return _check(st, "fa_backward_noalloc", check)
+
+
+def fa_forward_blocksparse(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, mask_heads,
+                           stream=None, check=True) -> int:
+    """Block-sparse forward; block_mask is a device uint8 [mask_heads, nt, nt]
+    buffer (nt = ceil(N / 128)), mask_heads 1 or H."""
+    st = _lib.fa_forward_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                     float(scale), int(bool(causal)), _ptr(block_mask),
+                                     int(mask_heads), _stream(stream))
+    return _check(st, "fa_forward_blocksparse", check)
+
+
+def fa_backward_blocksparse(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal,
+                            block_mask, mask_heads, workspace, workspace_bytes, stream=None,
+                            check=True) -> int:
+    st = _lib.fa_backward_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                      int(bool(causal)), _ptr(block_mask), int(mask_heads),
+                                      _ptr(workspace), int(workspace_bytes), _stream(stream))
+    return _check(st, "fa_backward_blocksparse", check)

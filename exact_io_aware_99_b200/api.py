@@ -32,10 +32,24 @@ def _check_inputs(*ts: torch.Tensor):
             raise ValueError("inputs must be contiguous CUDA tensors of one shape and dtype")
 
 
+def _block_mask(block_mask: torch.Tensor, H: int, N: int, device) -> Tuple[torch.Tensor, int]:
+    """Validate a block mask: bool/uint8 [nt, nt] or [Hm, nt, nt] (Hm = 1 or
+    H), nt = ceil(N / 128); returns a contiguous uint8 device copy and Hm."""
+    nt = (N + 127) // 128
+    m = block_mask if block_mask.dim() == 3 else block_mask.unsqueeze(0)
+    if m.dim() != 3 or tuple(m.shape[1:]) != (nt, nt) or m.shape[0] not in (1, H):
+        raise ValueError(f"block_mask must be [nt, nt] or [1 or H, nt, nt] with nt = {nt}")
+    m = m.to(device=device, dtype=torch.uint8).contiguous()
+    return m, int(m.shape[0])
+
+
 def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                       scale: Optional[float] = None, causal: bool = False,
-                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      block_mask: Optional[torch.Tensor] = None
                       ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """O and LSE.  With ``block_mask`` (bf16 only): block-sparse attention over
+    128 x 128 tiles, see ``fa_forward_blocksparse``."""
     _check_inputs(q, k, v)
     B, H, N, d = _dims(q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
@@ -43,14 +57,21 @@ def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
-    nat.fa_forward_ex(q, k, v, out, lse, B, H, N, d, scale, causal, _dtype_code(q))
+    if block_mask is not None:
+        m, mh = _block_mask(block_mask, H, N, q.device)
+        nat.fa_forward_blocksparse(q, k, v, out, lse, B, H, N, d, scale, causal, m, mh)
+    else:
+        nat.fa_forward_ex(q, k, v, out, lse, B, H, N, d, scale, causal, _dtype_code(q))
     return out, lse
 
 
 def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                        do: torch.Tensor, lse: torch.Tensor, scale: Optional[float] = None,
-                       causal: bool = False, workspace: Optional[torch.Tensor] = None
+                       causal: bool = False, workspace: Optional[torch.Tensor] = None,
+                       block_mask: Optional[torch.Tensor] = None
                        ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """dQ, dK, dV; ``block_mask`` as in ``attention_forward`` (same mask as the
+    forward)."""
     _check_inputs(q, k, v, o, do)
     B, H, N, d = _dims(q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
@@ -58,6 +79,11 @@ def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
     if workspace is None or workspace.numel() * workspace.element_size() < wbytes:
         workspace = torch.empty(wbytes, device=q.device, dtype=torch.uint8)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    nat.fa_backward_ex(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
-                       wbytes, _dtype_code(q))
+    if block_mask is not None:
+        m, mh = _block_mask(block_mask, H, N, q.device)
+        nat.fa_backward_blocksparse(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, causal,
+                                    m, mh, workspace, wbytes)
+    else:
+        nat.fa_backward_ex(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, causal,
+                           workspace, wbytes, _dtype_code(q))
     return dq, dk, dv

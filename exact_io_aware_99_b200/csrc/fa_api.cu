@@ -218,7 +218,7 @@ fa_status fa_forward_ex(const void* q, const void* k, const void* v, void* o, fl
     if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
     if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
     if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
-    e = fa::launch_fwd_sm100(tq, tk, tv, o, lse, BH, N, d, scale, cz, L);
+    e = fa::launch_fwd_sm100(tq, tk, tv, o, lse, BH, N, d, scale, cz, nullptr, L);
   }
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
@@ -226,6 +226,30 @@ fa_status fa_forward_ex(const void* q, const void* k, const void* v, void* o, fl
 fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int H, int N, int d, float scale, int causal, void* stream) {
   return fa_forward_ex(q, k, v, o, lse, B, H, N, d, scale, causal, FA_BF16, stream);
+}
+
+fa_status fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
+                                 float* lse, int B, int H, int N, int d, float scale, int causal,
+                                 const unsigned char* block_mask, int mask_heads, void* stream) {
+  if (!q || !k || !v || !o || !lse || !block_mask) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, FA_BF16);
+  if (st != FA_OK) return st;
+  if (mask_heads != 1 && mask_heads != H) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_MISALIGNED;
+  fa::Launch L;
+  st = device_context(stream, &L);
+  if (st != FA_OK) return st;
+  const int BH = B * H;
+  st = get_encoder();
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
+  const fa::BlockMaskArg bm{block_mask, mask_heads, H};
+  cudaError_t e = fa::launch_fwd_sm100(tq, tk, tv, o, lse, BH, N, d, scale, causal ? 1 : 0, &bm, L);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
 size_t fa_backward_workspace_size(int B, int H, int N, int d) {
@@ -274,7 +298,46 @@ fa_status fa_backward_ex(const void* q, const void* k, const void* v, const void
   if ((st = make_map(&tdo, dO, BH, N, d)) != FA_OK) return st;
   e = fa::launch_bwd_preprocess(o, dO, lse, dvec, lse2, BH, N, d, 1, L);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, d, scale, cz, L);
+  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, d, scale, cz, nullptr, L);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+fa_status fa_backward_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                                  const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                                  int B, int H, int N, int d, float scale, int causal,
+                                  const unsigned char* block_mask, int mask_heads,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !block_mask)
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, FA_BF16);
+  if (st != FA_OK) return st;
+  if (mask_heads != 1 && mask_heads != H) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  const WsLayout w = ws_layout(B, H, N, d);
+  if (!workspace || workspace_bytes < w.total ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FA_ERR_WORKSPACE;
+  fa::Launch L;
+  st = device_context(stream, &L);
+  if (st != FA_OK) return st;
+  const int BH = B * H;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dvec = reinterpret_cast<float*>(ws + w.dvec_off);
+  float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
+  st = get_encoder();
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&tdo, dO, BH, N, d)) != FA_OK) return st;
+  cudaError_t e = fa::launch_bwd_preprocess(o, dO, lse, dvec, lse2, BH, N, d, 1, L);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const fa::BlockMaskArg bm{block_mask, mask_heads, H};
+  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, d, scale,
+                           causal ? 1 : 0, &bm, L);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 

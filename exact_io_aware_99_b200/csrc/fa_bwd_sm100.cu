@@ -224,7 +224,7 @@ struct KvCfg : Shape<D> {
 // and writes its dS^T into [128+64h, 128+64h+32).
 constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvColDV = 256, kKvColDK = 384;
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -232,7 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ dvec,
                     const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dk,
                     __nv_bfloat16* __restrict__ dv, int N, int BH, int group, float scale,
-                    float scale_log2, WaitCtl ctl) {
+                    float scale_log2, const uint8_t* __restrict__ bmask, int mask_heads, int H,
+                    WaitCtl ctl) {
   using C = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -262,10 +263,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int Np = n_t * kT;
   // Key tile j and the query tiles [i_start, n_t) that see it, for work item
   // idx (group-major; j = 0 first: most query tiles when causal).
+  // With a block mask (BS) only the query tiles whose mask byte (i, j) is set
+  // are visited; next_i steps to the next of them.
+  const uint8_t* hmask = nullptr;  // this item's head's [n_t][n_t] mask (BS)
   auto decode = [&](int idx, int& bh, int& j, int& i_start, int& n_iter) {
     group_major(idx, n_t, BH, group, bh, j);
     i_start = CAUSAL ? j : 0;
     n_iter = n_t - i_start;
+    if (BS) {
+      hmask = bmask + static_cast<size_t>(mask_heads == 1 ? 0 : bh % H) * n_t * n_t;
+      n_iter = 0;
+      for (int i = i_start; i < n_t; ++i) n_iter += hmask[static_cast<size_t>(i) * n_t + j] != 0;
+    }
+  };
+  auto next_i = [&](int i, int j) -> int {
+    ++i;
+    if (BS)
+      while (i < n_t && hmask[static_cast<size_t>(i) * n_t + j] == 0) ++i;
+    return i;
   };
 
   if (threadIdx.x == 0) {
@@ -321,8 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         int bh, j, i_start, n_iter;
         decode(idx, bh, j, i_start, n_iter);
-        if (w > 0 &&
-            !mbar_wait(kv_empty, static_cast<uint32_t>(w - 1) & 1, abort, ctl, kSiteBwdProducer))
+        if (n_iter > 0) {
+        if (kv_issued > 0 && !mbar_wait(kv_empty, static_cast<uint32_t>(kv_issued - 1) & 1, abort,
+                                        ctl, kSiteBwdProducer))
           break;
         mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
 #pragma unroll
@@ -330,15 +346,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(&tm_k, kv_full, smem + C::K_OFF + b * C::BLK, b * 64, j * kT, bh);
           tma_load_3d(&tm_v, kv_full, smem + C::V_OFF + b * C::BLK, b * 64, j * kT, bh);
         }
-        kv_issued = w + 1;
+        ++kv_issued;
+        int ic = i_start - 1;  // query tile of the step
         for (int it = 0; it < n_iter; ++it, ++qr) {
+          ic = next_i(ic, j);
           const int st = static_cast<int>(qr & 1);
           const uint32_t u = qr >> 1;
           if (qr >= 2 && !mbar_wait(qdo_empty + st, (u - 1) & 1, abort, ctl, kSiteBwdProducer)) {
             ok = false;
             break;
           }
-          const int y = (i_start + it) * kT;
+          const int y = ic * kT;
           mbar_arrive_expect_tx(q_full + st, C::TILE + 1024);
 #pragma unroll
           for (int b = 0; b < C::NB; ++b)
@@ -355,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           last[st] = static_cast<int>(u);
         }
         if (!ok) break;
+        }  // n_iter > 0
         if (!producer_request_item(w, nxt_full, nxt_empty, nxt_resp, abort, ctl,
                                    kSiteBwdProducer, nxt_pending, nxt_pending_par))
           break;
@@ -434,14 +453,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dP^T_{i+1} overwrites dS^T_i in B: issued after dK_i, in order.
     bool ok = true;
     int idx = 0;
+    uint32_t kv_items = 0;  // items with at least one query tile (one K/V load each)
     for (int w = 0; ok; ++w) {
       if (!next_item(w, idx, kSiteBwdMma)) break;
       if (idx < 0) break;
       int bh, j, i_start;
       decode(idx, bh, j, i_start, n_iter);
+      if (n_iter == 0) continue;  // the block mask hides this key tile from every query
       s_done = dp_done = released = 0;
-      ok = wait_all(kv_full, static_cast<uint32_t>(w) & 1, abort, ctl, kSiteBwdMma) &&
-           issue_s(0) && issue_dp(0);
+      ok = wait_all(kv_full, kv_items & 1, abort, ctl, kSiteBwdMma) && issue_s(0) &&
+           issue_dp(0);
+      ++kv_items;
       for (int it = 0; ok && it < n_iter; ++it) {
         const uint32_t g = qbase + it;
         const int st = static_cast<int>(g & 1);
@@ -503,7 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t col_s = kKvColS + 64 * h;    // this half's S^T, then P^T
     const uint32_t col_dp = kKvColDP + 64 * h;  // this half's dP^T, then dS^T
-    uint32_t qbase = 0;  // query tiles of the previous items (barrier phases)
+    uint32_t qbase = 0;     // query tiles of the previous items (barrier phases)
+    uint32_t kv_items = 0;  // items with at least one query tile
     bool ok = true;
     int idx = 0;
     for (int w = 0; ok; ++w) {
@@ -513,8 +536,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode(idx, bh, j, i_start, n_iter);
       const int k_idx = j * kT + kr;
       const bool key_ok = k_idx < N;
+      if (n_iter == 0) {
+        // No query sees this key tile: dK = dV = 0 (block mask only).
+        const size_t row = (static_cast<size_t>(bh) * N + k_idx) * D;
+        if (key_ok)
+          for (int c = h; c < D / 8; c += 2) {
+            reinterpret_cast<uint4*>(dv + row)[c] = make_uint4(0u, 0u, 0u, 0u);
+            reinterpret_cast<uint4*>(dk + row)[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        continue;
+      }
+      int i = i_start - 1;  // query tile of the step
       for (int it = 0; it < n_iter; ++it) {
-        const int i = i_start + it;
+        i = next_i(i, j);
         const uint32_t g = qbase + it;
         const int st = static_cast<int>(g & 1);
         // LSE2 and D of this half's 64 queries, staged by the producer with
@@ -581,7 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // between the two warpgroups.  kv_done completes once per item; the
       // next item's first dV/dK MMAs (accumulate off) come after this
       // warpgroup's next P^T / dS^T, so the loads below are complete by then.
-      if (!wait_all(kv_done, static_cast<uint32_t>(w) & 1, abort, ctl, kSiteBwdEpilogue)) break;
+      if (!wait_all(kv_done, kv_items & 1, abort, ctl, kSiteBwdEpilogue)) break;
+      ++kv_items;
       tc_fence_after();
       const size_t row = (static_cast<size_t>(bh) * N + k_idx) * D;
       store_row_bf16<D>(lane_base + kKvColDV, 1.f, dv + row, key_ok, h);
@@ -627,13 +662,14 @@ struct QCfg : Shape<D> {
 // writes its dS (bf16 pairs) into [64h, 64h+32) of the same buffer.
 constexpr uint32_t kQColS = 0, kQColDP = 256, kQColDQ = 384;
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ dvec,
                   const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dq, int N, int BH,
-                  int group, float scale, float scale_log2, WaitCtl ctl) {
+                  int group, float scale, float scale_log2, const uint8_t* __restrict__ bmask,
+                  int mask_heads, int H, WaitCtl ctl) {
   using C = QCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -663,11 +699,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int Np = n_t * kT;
   // Query tile i and the key tiles it sees for work item idx (group-major,
   // longest query tiles first when causal).
+  // With a block mask (BS) only the key tiles whose mask byte (i, j) is set
+  // are visited; next_j steps to the next of them.
+  const uint8_t* hrow = nullptr;  // this item's mask row (BS)
   auto decode = [&](int idx, int& bh, int& i, int& n_kv) {
     int t;
     group_major(idx, n_t, BH, group, bh, t);
     i = n_t - 1 - t;
     n_kv = CAUSAL ? i + 1 : n_t;
+    if (BS) {
+      hrow = bmask + (static_cast<size_t>(mask_heads == 1 ? 0 : bh % H) * n_t + i) * n_t;
+      const int jend = n_kv;
+      n_kv = 0;
+      for (int j = 0; j < jend; ++j) n_kv += hrow[j] != 0;
+    }
+  };
+  auto next_j = [&](int j) -> int {
+    ++j;
+    if (BS)
+      while (j < n_t && hrow[j] == 0) ++j;
+    return j;
   };
 
   if (threadIdx.x == 0) {
@@ -731,8 +782,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         int bh, i, n_kv;
         decode(idx, bh, i, n_kv);
-        if (it > 0 &&
-            !mbar_wait(q_empty, static_cast<uint32_t>(it - 1) & 1, abort, ctl, kSiteBwdProducer))
+        if (n_kv > 0) {
+        if (q_issued > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(q_issued - 1) & 1, abort,
+                                       ctl, kSiteBwdProducer))
           break;
         mbar_arrive_expect_tx(q_full, 2 * C::TILE);
 #pragma unroll
@@ -740,8 +792,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + b * C::BLK, b * 64, i * kT, bh);
           tma_load_3d(&tm_do, q_full, smem + C::DO_OFF + b * C::BLK, b * 64, i * kT, bh);
         }
-        q_issued = it + 1;
+        ++q_issued;
+        int jt = -1;  // key tile of the step
         for (int jj = 0; jj < n_kv; ++jj, ++kr) {
+          jt = next_j(jt);
           const int sk = static_cast<int>(kr % C::NK), sv = static_cast<int>(kr % C::NV);
           const uint32_t uk = kr / C::NK, uv = kr / C::NV;
           if (kr >= C::NK &&
@@ -753,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int b = 0; b < C::NB; ++b)
             tma_load_3d(&tm_k, k_full + sk, smem + C::K_OFF + sk * C::TILE + b * C::BLK, b * 64,
-                        jj * kT, bh);
+                        jt * kT, bh);
           last_k[sk] = static_cast<int>(uk);
           if (kr >= C::NV &&
               !mbar_wait(v_empty + sv, (uv - 1) & 1, abort, ctl, kSiteBwdProducer)) {
@@ -764,10 +818,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int b = 0; b < C::NB; ++b)
             tma_load_3d(&tm_v, v_full + sv, smem + C::V_OFF + sv * C::TILE + b * C::BLK, b * 64,
-                        jj * kT, bh);
+                        jt * kT, bh);
           last_v[sv] = static_cast<int>(uv);
         }
         if (!ok) break;
+        }  // n_kv > 0
         if (!producer_request_item(it, nxt_full, nxt_empty, nxt_resp, abort, ctl,
                                    kSiteBwdProducer, nxt_pending, nxt_pending_par))
           break;
@@ -852,14 +907,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // softmax has read it.
     bool ok = true;
     int idx = 0;
+    uint32_t q_items = 0;  // items with at least one key tile (one Q load each)
     for (int it = 0; ok; ++it) {
       if (!next_item(it, idx, kSiteBwdMma)) break;
       if (idx < 0) break;
       int bh, i;
       decode(idx, bh, i, n_kv);
+      if (n_kv == 0) continue;  // the block mask hides every key from this query tile
       released = s_done = dp_done = 0;
-      ok = wait_all(q_full, static_cast<uint32_t>(it) & 1, abort, ctl, kSiteBwdMma) &&
-           issue_s(0) && issue_dp(0);
+      ok = wait_all(q_full, q_items & 1, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
+      ++q_items;
       if (ok && n_kv > 1) ok = issue_s(1);
       for (int jj = 0; ok && jj < n_kv; ++jj) {
         const uint32_t g = kbase + jj;
@@ -905,7 +962,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2;
     const int qr = threadIdx.x & 127;  // query row == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    uint32_t kbase = 0;  // key tiles of the previous items (S buffer numbering)
+    uint32_t kbase = 0;    // key tiles of the previous items (S buffer numbering)
+    uint32_t q_items = 0;  // items with at least one key tile
     bool ok = true;
     int idx = 0;
     for (int it = 0; ok; ++it) {
@@ -914,9 +972,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       int bh, i, n_kv;
       decode(idx, bh, i, n_kv);
       const int q_idx = i * kT + qr;
+      if (n_kv == 0) {
+        // These queries see no key: dQ = 0 (block mask only).
+        if (q_idx < N) {
+          uint4* row = reinterpret_cast<uint4*>(dq + (static_cast<size_t>(bh) * N + q_idx) * D);
+          for (int c = h; c < D / 8; c += 2) row[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
       const float my_l2 = lse2[static_cast<size_t>(bh) * Np + q_idx];  // +inf past N
       const float my_d = dvec[static_cast<size_t>(bh) * Np + q_idx];
+      int jt = -1;  // key tile of the step
       for (int jj = 0; jj < n_kv; ++jj) {
+        jt = next_j(jt);
         const uint32_t g = kbase + jj;
         const uint32_t col_s = kQColS + (g & 1) * kT + 64 * h;
         if (!wait_all(s_full + (g & 1), (g >> 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
@@ -928,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + col_s, sv[0]);
         tmem_ld32(lane_base + col_s + 32, sv[1]);
         tmem_wait_ld();
-        const int k0 = jj * kT + 64 * h;  // first key of this half
+        const int k0 = jt * kT + 64 * h;  // first key of this half
         // keys k visible to this query: k <= q_idx (causal) and k < N
         const int lim = min(N, CAUSAL ? q_idx + 1 : N) - k0;
         float p[64];
@@ -963,7 +1031,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dq_done completes once per item; the next item's first dQ MMA
       // (accumulate off) comes after this warpgroup's next dS, so the loads
       // below are complete by then.
-      if (!wait_all(dq_done, static_cast<uint32_t>(it) & 1, abort, ctl, kSiteBwdEpilogue)) break;
+      if (!wait_all(dq_done, q_items & 1, abort, ctl, kSiteBwdEpilogue)) break;
+      ++q_items;
       tc_fence_after();
       store_row_bf16<D>(lane_base + kQColDQ, scale, dq + (static_cast<size_t>(bh) * N + q_idx) * D,
                         q_idx < N, h);
@@ -992,17 +1061,18 @@ inline int heads_per_group(long long per_head_bytes, int BH, bool causal) {
   return g < 1 ? 1 : (g > BH ? BH : g);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool BS>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& tdo, const float* dvec, const float* lse2, void* dq,
-                   void* dk, void* dv, int BH, int N, float scale, const Launch& L) {
+                   void* dk, void* dv, int BH, int N, float scale, const BlockMaskArg& bm,
+                   const Launch& L) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, CAUSAL>,
+    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, CAUSAL, BS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          KvCfg<D>::SMEM);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_dq_kernel<D, CAUSAL>,
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D, CAUSAL, BS>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, QCfg<D>::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
@@ -1010,21 +1080,38 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   const int n_t = (N + kT - 1) / kT;
   const long long blocks = static_cast<long long>(BH) * n_t;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  // Heads per group: a group's Q, K, V, dO (bf16, 8 N d bytes per head)
-  // within ~48 MB of the 126 MB L2.
   const int group = heads_per_group(4LL * N * D, BH, CAUSAL);
   const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};
-  bwd_dkdv_kernel<D, CAUSAL>
+  bwd_dkdv_kernel<D, CAUSAL, BS>
       <<<static_cast<unsigned>(blocks), kThreads, KvCfg<D>::SMEM, L.stream>>>(
           tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dk),
-          static_cast<__nv_bfloat16*>(dv), N, BH, group, scale, scale_log2, ctl);
+          static_cast<__nv_bfloat16*>(dv), N, BH, group, scale, scale_log2, bm.mask,
+          bm.mask_heads, bm.H, ctl);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D, CAUSAL><<<static_cast<unsigned>(blocks), kThreads, QCfg<D>::SMEM, L.stream>>>(
-      tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dq), N, BH, group, scale,
-      scale_log2, ctl);
+  bwd_dq_kernel<D, CAUSAL, BS>
+      <<<static_cast<unsigned>(blocks), kThreads, QCfg<D>::SMEM, L.stream>>>(
+          tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dq), N, BH, group, scale,
+          scale_log2, bm.mask, bm.mask_heads, bm.H, ctl);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& tdo, const float* dvec, const float* lse2, void* dq,
+                     void* dk, void* dv, int BH, int N, float scale, int causal,
+                     const BlockMaskArg* bm, const Launch& L) {
+  const BlockMaskArg none{nullptr, 1, 1};
+  if (bm && bm->mask)
+    return causal ? launch<D, true, true>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale,
+                                          *bm, L)
+                  : launch<D, false, true>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale,
+                                           *bm, L);
+  return causal ? launch<D, true, false>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale,
+                                         none, L)
+                : launch<D, false, false>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale,
+                                          none, L);
 }
 
 }  // namespace bwd
@@ -1032,21 +1119,20 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tdo, const float* dvec, const float* lse2,
                              void* dq, void* dk, void* dv, int BH, int N, int d, float scale,
-                             int causal, const Launch& L) {
-#define FA_BWD_CASE(DD)                                                                       \
-  case DD:                                                                                    \
-    return causal ? bwd::launch<DD, true>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N,     \
-                                          scale, L)                                           \
-                  : bwd::launch<DD, false>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N,    \
-                                           scale, L);
+                             int causal, const BlockMaskArg* bm, const Launch& L) {
   switch (d) {
-    FA_BWD_CASE(64)
-    FA_BWD_CASE(80)
-    FA_BWD_CASE(128)
+    case 64:
+      return bwd::launch_d<64>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale, causal, bm,
+                               L);
+    case 80:
+      return bwd::launch_d<80>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale, causal, bm,
+                               L);
+    case 128:
+      return bwd::launch_d<128>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale, causal,
+                                bm, L);
     default:
       return cudaErrorInvalidValue;
   }
-#undef FA_BWD_CASE
 }
 
 }  // namespace fa

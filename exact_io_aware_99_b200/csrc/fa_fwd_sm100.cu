@@ -120,12 +120,60 @@ __device__ __forceinline__ void decode_item(int idx, int n_t, int BH, int group,
   }
 }
 
-template <int D, bool CAUSAL>
+// Key tiles of one work item when a block mask is given (block-sparse
+// attention): tile x of the pair (query tile qt[x]) sees key tile j when the
+// tile exists, j <= qt[x] if causal, and the mask byte (qt[x], j) is set.
+// The pair visits the union of its two tiles' key tiles; a tile that does not
+// see a visited key tile treats that step as fully masked.
+template <bool CAUSAL>
+struct ItemTiles {
+  const uint8_t* row[2];  // mask rows of the two query tiles
+  int qt[2];
+  bool has[2];
+  int n_t;
+  __device__ __forceinline__ bool active(int x, int j) const {
+    return has[x] && (!CAUSAL || j <= qt[x]) && row[x][j] != 0;
+  }
+  __device__ __forceinline__ bool any(int j) const { return active(0, j) || active(1, j); }
+  // First visited key tile after j (n_t when there is none).
+  __device__ __forceinline__ int next(int j) const {
+    do {
+      ++j;
+    } while (j < n_t && !any(j));
+    return j;
+  }
+};
+
+// Steps of a work item and, with a block mask, the tiles it visits.  Dense:
+// tile x visits key tiles [0, n_x[x]); block-sparse: both tiles step through
+// the union of visited key tiles (n_x[1] = 0 when tile B lies past N).
+template <bool CAUSAL, bool BS>
+__device__ __forceinline__ void item_plan(int idx, int n_t, int BH, int group, int H,
+                                          const uint8_t* bmask, int mask_heads, int& bh,
+                                          int& pair, int (&n_x)[2], ItemTiles<CAUSAL>& it) {
+  decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+  if (BS) {
+    const int hm = mask_heads == 1 ? 0 : bh % H;
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      it.qt[x] = 2 * pair + x;
+      it.has[x] = it.qt[x] < n_t;
+      it.row[x] = bmask + (static_cast<size_t>(hm) * n_t + (it.has[x] ? it.qt[x] : 0)) * n_t;
+    }
+    it.n_t = n_t;
+    int steps = 0;
+    for (int j = it.next(-1); j < n_t; j = it.next(j)) ++steps;
+    n_x[0] = steps;
+    n_x[1] = it.has[1] ? steps : 0;
+  }
+}
+
+template <int D, bool CAUSAL, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                float* __restrict__ lse, int N, int BH, int group, float scale_log2,
-               WaitCtl ctl) {
+               const uint8_t* __restrict__ bmask, int mask_heads, int H, WaitCtl ctl) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -230,11 +278,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (idx < 0) break;
         }
         int bh, pair, n_x[2];
-        decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+        ItemTiles<CAUSAL> tiles;
+        item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
         const int n_max = max(n_x[0], n_x[1]);
+        if (n_max > 0) {
         // Q of this item replaces the previous item's once its S MMAs are done.
-        if (i > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(i - 1) & 1, abort, ctl,
-                                kSiteFwdProducer))
+        if (q_issued > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(q_issued - 1) & 1, abort,
+                                       ctl, kSiteFwdProducer))
           break;
         const int nq = n_x[1] > 0 ? 2 : 1;
         mbar_arrive_expect_tx(q_full, nq * C::TILE);
@@ -243,8 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int b = 0; b < C::NB; ++b)
             tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + x * C::TILE + b * C::BLK, b * 64,
                         (2 * pair + x) * kBM, bh);
-        q_issued = i + 1;
+        ++q_issued;
+        int jt = -1;  // key tile of the step
         for (int j = 0; j < n_max; ++j, ++kv) {
+          jt = BS ? tiles.next(jt) : j;
           const int s = static_cast<int>(kv % C::NST);
           const uint32_t u = kv / C::NST;
           if (kv >= C::NST && !mbar_wait(k_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer)) {
@@ -255,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int b = 0; b < C::NB; ++b)
             tma_load_3d(&tm_k, k_full + s, smem + C::K_OFF + s * C::TILE + b * C::BLK, b * 64,
-                        j * kBN, bh);
+                        jt * kBN, bh);
           last_k[s] = static_cast<int>(u);
           if (kv >= C::NST && !mbar_wait(v_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer)) {
             ok = false;
@@ -265,10 +317,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int b = 0; b < C::NB; ++b)
             tma_load_3d(&tm_v, v_full + s, smem + C::V_OFF + s * C::TILE + b * C::BLK, b * 64,
-                        j * kBN, bh);
+                        jt * kBN, bh);
           last_v[s] = static_cast<int>(u);
         }
         if (!ok) break;
+        }  // n_max > 0
         // Ask for the next item now, while this one's MMAs and softmax run.
         const int sl1 = (i + 1) & 1;
         const uint32_t u1 = static_cast<uint32_t>(i >> 1);
@@ -343,14 +396,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     bool ok = true;
     int idx = 0;
+    uint32_t q_items = 0;  // items with at least one step (one Q load each)
     for (int i = 0; ok; ++i) {
       if (!next_item(i, idx, kSiteFwdMma)) break;
       if (idx < 0) break;
       int bh, pair, n_x[2];
-      decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+      ItemTiles<CAUSAL> tiles;
+      item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
       const int n_max = max(n_x[0], n_x[1]);
+      if (n_max == 0) continue;  // block mask hides the whole item
       const int r0 = static_cast<int>(kv_base);
-      ok = wait_all(q_full, static_cast<uint32_t>(i) & 1, abort, ctl, kSiteFwdMma) && wait_k(r0);
+      ok = wait_all(q_full, q_items & 1, abort, ctl, kSiteFwdMma) && wait_k(r0);
+      ++q_items;
       if (!ok) break;
       tc_fence_after();
       for (int x = 0; x < 2; ++x)
@@ -406,12 +463,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!next_item(i, idx, kSiteFwdSoftmax)) break;
       if (idx < 0) break;
       int bh, pair, n_x[2];
-      decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+      ItemTiles<CAUSAL> tiles;
+      item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
       const int n_kv = n_x[x];
-      const int q_idx = (2 * pair + x) * kBM + r;
+      const int qt_x = 2 * pair + x;
+      const int q_idx = qt_x * kBM + r;
+      if (n_kv == 0) {
+        // The block mask hides every key from this tile: O = 0, LSE = -inf.
+        // (Dense launches only get here for a tile past N: nothing to write.)
+        if (q_idx < N) {
+          uint4* orow = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+          lse[static_cast<size_t>(bh) * N + q_idx] = -INFINITY;
+        }
+        continue;
+      }
       float m = -INFINITY;  // reference max, base-2 scaled units
       float l = 0.f;
+      int jt = -1;          // key tile of the step
       for (int j = 0; j < n_kv; ++j) {
+        jt = BS ? tiles.next(jt) : j;
         if (!wait_all(s_full + x, (s_base + j) & 1, abort, ctl, kSiteFwdSoftmax)) {
           ok = false;
           break;
@@ -437,10 +509,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             s[96 + c] = __uint_as_float(t1[c]);
           }
         }
-        const int kv0 = j * kBN;
-        const bool diag = CAUSAL && (j == n_kv - 1);
-        const bool masked = diag || kv0 + kBN > N;
-        const int lim = masked ? min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN) : kBN;
+        const int kv0 = jt * kBN;
+        const bool act = !BS || tiles.active(x, jt);  // false: the mask hides the whole step
+        const bool diag = CAUSAL && (BS ? jt == qt_x : j == n_kv - 1);
+        const bool masked = !act || diag || kv0 + kBN > N;
+        const int lim =
+            !act ? 0 : (masked ? min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN) : kBN);
         if (masked) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
@@ -514,7 +588,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && n_kv > 0 &&
           wait_all(o_done + x, (s_base + n_kv - 1) & 1, abort, ctl, kSiteFwdEpilogue)) {
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        // l = 0 only for a row the block mask hides completely: O = 0.
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
         const bool valid = q_idx < N;
         uint4* orow = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
 #pragma unroll
@@ -533,7 +608,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (valid)
-          lse[static_cast<size_t>(bh) * N + q_idx] = (m + __log2f(l)) * 0.69314718055994531f;
+          lse[static_cast<size_t>(bh) * N + q_idx] =
+              l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         // The next item's first P V (accumulate off) overwrites O_x only
         // after this warpgroup's next P, so the loads above are complete.
         tc_fence_before();
@@ -552,20 +628,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool BS>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                   float* lse, int BH, int N, float scale, const Launch& L) {
+                   float* lse, int BH, int N, float scale, const BlockMaskArg& bm,
+                   const Launch& L) {
   using C = Cfg<D>;
   static bool configured = false;
   if (!configured) {
     // The register split above assumes the kernel was compiled to exactly
     // kLaunchRegs per thread; with fewer, the increase would wait forever.
     cudaFuncAttributes fattr;
-    cudaError_t e = cudaFuncGetAttributes(&fattr, fwd_kernel<D, CAUSAL>);
+    cudaError_t e = cudaFuncGetAttributes(&fattr, fwd_kernel<D, CAUSAL, BS>);
     if (e != cudaSuccess) return e;
     if (fattr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(fwd_kernel<D, CAUSAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM);
+    e = cudaFuncSetAttribute(fwd_kernel<D, CAUSAL, BS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -585,26 +662,36 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};
-  fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
-      tq, tk, tv, static_cast<__nv_bfloat16*>(o), lse, N, BH, group, scale_log2, ctl);
+  fwd_kernel<D, CAUSAL, BS><<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
+      tq, tk, tv, static_cast<__nv_bfloat16*>(o), lse, N, BH, group, scale_log2, bm.mask,
+      bm.mask_heads, bm.H, ctl);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     void* o, float* lse, int BH, int N, float scale, int causal,
+                     const BlockMaskArg* bm, const Launch& L) {
+  const BlockMaskArg none{nullptr, 1, 1};
+  if (bm && bm->mask)
+    return causal ? launch<D, true, true>(tq, tk, tv, o, lse, BH, N, scale, *bm, L)
+                  : launch<D, false, true>(tq, tk, tv, o, lse, BH, N, scale, *bm, L);
+  return causal ? launch<D, true, false>(tq, tk, tv, o, lse, BH, N, scale, none, L)
+                : launch<D, false, false>(tq, tk, tv, o, lse, BH, N, scale, none, L);
 }
 
 }  // namespace fwd
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              void* o, float* lse, int BH, int N, int d, float scale, int causal,
-                             const Launch& L) {
+                             const BlockMaskArg* bm, const Launch& L) {
   switch (d) {
     case 64:
-      return causal ? fwd::launch<64, true>(tq, tk, tv, o, lse, BH, N, scale, L)
-                    : fwd::launch<64, false>(tq, tk, tv, o, lse, BH, N, scale, L);
+      return fwd::launch_d<64>(tq, tk, tv, o, lse, BH, N, scale, causal, bm, L);
     case 80:
-      return causal ? fwd::launch<80, true>(tq, tk, tv, o, lse, BH, N, scale, L)
-                    : fwd::launch<80, false>(tq, tk, tv, o, lse, BH, N, scale, L);
+      return fwd::launch_d<80>(tq, tk, tv, o, lse, BH, N, scale, causal, bm, L);
     case 128:
-      return causal ? fwd::launch<128, true>(tq, tk, tv, o, lse, BH, N, scale, L)
-                    : fwd::launch<128, false>(tq, tk, tv, o, lse, BH, N, scale, L);
+      return fwd::launch_d<128>(tq, tk, tv, o, lse, BH, N, scale, causal, bm, L);
     default:
       return cudaErrorInvalidValue;
   }

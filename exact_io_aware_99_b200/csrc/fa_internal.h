@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstddef>
+#include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -51,12 +52,21 @@ inline long long l2_group_bytes(int causal) {
   return static_cast<long long>(causal ? FA_L2_GROUP_MB : FA_L2_GROUP_MB_NONCAUSAL) << 20;
 }
 
+// Block mask of block-sparse attention: mask[(hm * n_t + i) * n_t + j] != 0
+// lets query tile i (128 rows) see key tile j, n_t = ceil(N / 128); hm = 0
+// when mask_heads == 1 (one mask for every head), else hm = (b * H + h) % H.
+struct BlockMaskArg {
+  const uint8_t* mask;  // device pointer; nullptr = dense
+  int mask_heads;       // 1 or H
+  int H;                // heads per batch entry
+};
+
 // --- bf16 tensor-core path (fa_fwd_sm100.cu, fa_bwd_sm100.cu) -------------
 // Tensor maps describe a [BH, N, d] bf16 tensor as 3-D {d, N, BH} with a
 // {64, 128, 1} box and 128-byte swizzle.
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              void* o, float* lse, int BH, int N, int d, float scale, int causal,
-                             const Launch& L);
+                             const BlockMaskArg* bm, const Launch& L);
 
 // Backward: the dK/dV kernel then the dQ kernel, both in stream order.
 // dvec and lse2 are the preprocess outputs ([BH, Np] fp32, Np = N rounded up
@@ -64,7 +74,7 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tdo, const float* dvec, const float* lse2,
                              void* dq, void* dk, void* dv, int BH, int N, int d, float scale,
-                             int causal, const Launch& L);
+                             int causal, const BlockMaskArg* bm, const Launch& L);
 
 // --- helpers shared by both dtypes (fa_simt.cu) ---------------------------
 // D = rowsum(dO o O) (fp32, padded rows = 0) and, when lse2 is non-null,

@@ -147,6 +147,47 @@ FA_API fa_status fa_backward_ex(const void* q, const void* k, const void* v,
                          fa_dtype dtype, void* stream);
 
 /*
+ * fa_forward_blocksparse -- bf16 forward of block-sparse attention: the
+ * combination of FlashAttention-2 with a block sparsity pattern described in
+ * "FlashAttention-2: Faster Attention with Better Parallelism and Work
+ * Partitioning" (review page), answer on combining it with sparse / hybrid
+ * attention, section 3 (1) "Sparse FlashAttention" (a pattern defined on
+ * blocks matched to the kernel's tiles; only the important blocks are
+ * processed), and the limitations answer, section 2 (3) (dense global plus
+ * sparse local attention).
+ *   block_mask  device pointer, uint8 [mask_heads, nt, nt] with
+ *               nt = ceil(N / 128): byte (h, I, J) != 0 lets query rows
+ *               128 I .. 128 I + 127 see keys 128 J .. 128 J + 127 of head h.
+ *               Key tiles a query tile may not see are never loaded.
+ *   mask_heads  1 (one mask for every head) or H (head h of every batch
+ *               entry uses mask h).
+ *   causal      applied on top of the mask (query i sees keys j <= i).
+ * A query row that sees no key at all gets O = 0 and LSE = -inf.  The mask
+ * must stay unchanged until the call's kernels have run.  Other arguments and
+ * errors as fa_forward; a null block_mask or mask_heads not in {1, H} is
+ * FA_ERR_INVALID_ARG.
+ */
+FA_API fa_status fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int H, int N, int d, float scale,
+                                        int causal, const unsigned char* block_mask,
+                                        int mask_heads, void* stream);
+
+/*
+ * fa_backward_blocksparse -- bf16 backward of fa_forward_blocksparse: the
+ * gradients of the masked softmax attention (hidden entries have P = 0, so
+ * they pass no gradient).  Key tiles no query may see get dK = dV = 0; query
+ * rows that see no key get dQ = 0.  Arguments as fa_backward plus the same
+ * block_mask / mask_heads as the forward; the workspace is sized by
+ * fa_backward_workspace_size.
+ */
+FA_API fa_status fa_backward_blocksparse(const void* q, const void* k, const void* v,
+                                         const void* o, const void* dO, const float* lse,
+                                         void* dq, void* dk, void* dv, int B, int H, int N,
+                                         int d, float scale, int causal,
+                                         const unsigned char* block_mask, int mask_heads,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_backward_noalloc -- the bf16 backward of fa_backward, for callers that
  * cannot allocate device memory or hand over a workspace: code whose device
  * memory is entirely owned by another allocator, plugins and callbacks that
