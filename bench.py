@@ -180,13 +180,24 @@ def run_ours(args, peaks, peak_kind):
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     scale, causal = w.scale, w.causal
+    mask_np = workloads.block_mask(w)
+    if mask_np is not None:
+        mask = torch.from_numpy(mask_np.astype("uint8")).to(dev).contiguous()
+        mh = int(mask.shape[0])
 
-    def fwd():
-        fa.fa_forward(q, k, v, o, lse, B, H, N, d, scale, causal, sp)
+        def fwd():
+            fa.fa_forward_blocksparse(q, k, v, o, lse, B, H, N, d, scale, causal, mask, mh, sp)
 
-    def bwd():
-        fa.fa_backward(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, causal, wsbuf, wbytes,
-                       sp)
+        def bwd():
+            fa.fa_backward_blocksparse(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale,
+                                       causal, mask, mh, wsbuf, wbytes, sp)
+    else:
+        def fwd():
+            fa.fa_forward(q, k, v, o, lse, B, H, N, d, scale, causal, sp)
+
+        def bwd():
+            fa.fa_backward(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, causal, wsbuf,
+                           wbytes, sp)
 
     def barrier():
         if ws > 1:
@@ -236,8 +247,7 @@ def run_ours(args, peaks, peak_kind):
         total_ms = float(t.item())
     ms_step = total_ms / args.steps
 
-    flops_f = perf.fwd_flops(B, H, N, d, causal)
-    flops_b = perf.bwd_flops(B, H, N, d, causal)
+    flops_f, flops_b = step_flop_counts(w)
     step_flops = flops_f + flops_b
     value = ws * step_flops / (ms_step * 1e-3) / 1e12
 
@@ -308,7 +318,10 @@ def run_ours(args, peaks, peak_kind):
                    "causal": causal, "passes": "fwd+bwd",
                    "l2": "working set ~%.2f GB > 126 MB L2 (no flush needed)"
                          % ((7 * B * H * N * d * 2 + wbytes) / 1e9),
-                   "parallelism": f"{ws} independent replicas" if ws > 1 else "single GPU"},
+                   "parallelism": f"{ws} independent replicas" if ws > 1 else "single GPU",
+                   **({"block_mask": w.mask,
+                       "visible_fraction": round(float(mask_np.mean()), 4)}
+                      if mask_np is not None else {})},
         "fwd_tflops": round(fwd_tf, 3), "bwd_tflops": round(bwd_tf, 3),
         "fwd_frac_of_peak": round(fwd_tf / peak, 4), "bwd_frac_of_peak": round(bwd_tf / peak, 4),
         "frac_of_peak": round(value / ws / peak, 4),
@@ -331,19 +344,42 @@ def run_ours(args, peaks, peak_kind):
 
 # ------------------------------------------------------------- CPU oracle
 
+def step_flop_counts(w, B=None, H=None):
+    """Algorithmic forward and backward FLOPs of one step of workload w
+    (visible pairs only for a block-sparse workload)."""
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    m = workloads.block_mask(w)
+    if m is not None:
+        return (perf.fwd_flops_masked(B, H, w.N, w.d, w.causal, m),
+                perf.bwd_flops_masked(B, H, w.N, w.d, w.causal, m))
+    return perf.fwd_flops(B, H, w.N, w.d, w.causal), perf.bwd_flops(B, H, w.N, w.d, w.causal)
+
+
+def oracle_head_step(w, x, h):
+    """Forward and backward of head h of x on the fp64 oracle (the
+    block-sparse oracle for a block-sparse workload)."""
+    import oracle
+    qh, kh, vh, doh = (x[n][0, h] for n in ("q", "k", "v", "do"))
+    m = workloads.block_mask(w)
+    if m is not None:
+        from oracle.block_sparse import block_sparse_backward, block_sparse_forward
+        block_sparse_forward(qh, kh, vh, w.scale, m, w.causal)
+        block_sparse_backward(qh, kh, vh, doh, w.scale, m, w.causal)
+    else:
+        oracle.attention_forward(qh, kh, vh, w.scale, w.causal)
+        oracle.attention_backward(qh, kh, vh, doh, w.scale, w.causal)
+
+
 def cpu_baseline(w, seconds: float):
     """The fp64 oracle (as it stands) on a bounded sample of the workload:
     whole heads, forward and backward, until about ``seconds`` of CPU work."""
-    import oracle
     x = workloads.make_inputs(w, with_grad_out=True, B=1)
     cores = os.cpu_count() or 1
     n_heads, flops, t0 = 0, 0.0, time.perf_counter()
-    per_head = perf.fwd_flops(1, 1, w.N, w.d, w.causal) + perf.bwd_flops(1, 1, w.N, w.d, w.causal)
+    per_head = sum(step_flop_counts(w, B=1, H=1))
     while True:
-        h = n_heads % w.H
-        qh, kh, vh, doh = (x[n][0, h] for n in ("q", "k", "v", "do"))
-        oracle.attention_forward(qh, kh, vh, w.scale, w.causal)
-        oracle.attention_backward(qh, kh, vh, doh, w.scale, w.causal)
+        oracle_head_step(w, x, n_heads % w.H)
         n_heads += 1
         flops += per_head
         if time.perf_counter() - t0 >= seconds:
@@ -358,16 +394,12 @@ def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return None
-    import oracle
     w = workloads.WORKLOADS[args.workload]
     x = workloads.make_inputs(w, with_grad_out=True, B=1)
-    per_head = perf.fwd_flops(1, 1, w.N, w.d, w.causal) + perf.bwd_flops(1, 1, w.N, w.d, w.causal)
+    per_head = sum(step_flop_counts(w, B=1, H=1))
 
     def step(i):
-        h = i % w.H
-        qh, kh, vh, doh = (x[n][0, h] for n in ("q", "k", "v", "do"))
-        oracle.attention_forward(qh, kh, vh, w.scale, w.causal)
-        oracle.attention_backward(qh, kh, vh, doh, w.scale, w.causal)
+        oracle_head_step(w, x, i % w.H)
 
     for i in range(args.warmup):
         step(i)

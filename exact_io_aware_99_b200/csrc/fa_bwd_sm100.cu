@@ -109,6 +109,36 @@ __device__ __forceinline__ void group_major(int idx, int n_tiles, int BH, int gr
   bh = g * group + (r - t * gh);
 }
 
+// Tiles visited under a block mask, as 32-tile ballot words (see TileCursor;
+// all lanes of a converged warp call word()).
+// ColTiles: query tiles i in [lo, n_t) whose mask byte (i, j) is set -- the
+// query tiles that see key tile j (dK/dV kernel).
+struct ColTiles {
+  const uint8_t* m;  // [n_t][n_t] mask of the head
+  int n_t, j, lo;
+  __device__ __forceinline__ uint32_t word(int w) const {
+    const int i = 32 * w + lane_id();
+    return __ballot_sync(0xffffffffu,
+                         i >= lo && i < n_t && m[static_cast<size_t>(i) * n_t + j] != 0);
+  }
+};
+// RowTiles: key tiles j < hi whose mask byte (i, j) is set -- the key tiles
+// query tile i sees (dQ kernel).
+struct RowTiles {
+  const uint8_t* r;  // mask row of query tile i
+  int n_t, hi;
+  __device__ __forceinline__ uint32_t word(int w) const {
+    const int j = 32 * w + lane_id();
+    return __ballot_sync(0xffffffffu, j < hi && r[j] != 0);
+  }
+};
+template <class Tiles>
+__device__ __forceinline__ int count_tiles(const Tiles& t) {
+  int c = 0;
+  for (int w = 0; w < (t.n_t + 31) / 32; ++w) c += __popc(t.word(w));
+  return c;
+}
+
 // Store one row of a tile from TMEM columns [taddr, taddr + D) (fp32, times
 // `mul`) to global memory as bf16, 16 columns per step; the steps alternate
 // between the two softmax warpgroups (h = 0, 1).
@@ -264,23 +294,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Key tile j and the query tiles [i_start, n_t) that see it, for work item
   // idx (group-major; j = 0 first: most query tiles when causal).
   // With a block mask (BS) only the query tiles whose mask byte (i, j) is set
-  // are visited; next_i steps to the next of them.
-  const uint8_t* hmask = nullptr;  // this item's head's [n_t][n_t] mask (BS)
+  // are visited (`tiles`, walked with a TileCursor).  Every role calls this
+  // with its whole (converged) warp.
+  ColTiles tiles{bmask, n_t, 0, 0};
   auto decode = [&](int idx, int& bh, int& j, int& i_start, int& n_iter) {
     group_major(idx, n_t, BH, group, bh, j);
     i_start = CAUSAL ? j : 0;
     n_iter = n_t - i_start;
     if (BS) {
-      hmask = bmask + static_cast<size_t>(mask_heads == 1 ? 0 : bh % H) * n_t * n_t;
-      n_iter = 0;
-      for (int i = i_start; i < n_t; ++i) n_iter += hmask[static_cast<size_t>(i) * n_t + j] != 0;
+      tiles = ColTiles{bmask + static_cast<size_t>(mask_heads == 1 ? 0 : bh % H) * n_t * n_t,
+                       n_t, j, i_start};
+      n_iter = count_tiles(tiles);
     }
-  };
-  auto next_i = [&](int i, int j) -> int {
-    ++i;
-    if (BS)
-      while (i < n_t && hmask[static_cast<size_t>(i) * n_t + j] == 0) ++i;
-    return i;
   };
 
   if (threadIdx.x == 0) {
@@ -315,78 +340,86 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the loop (it reads the block mask with all lanes);
+    // the elected lane issues the copies and the next-item requests.
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      int last[2] = {-1, -1};
-      int kv_issued = 0;
-      int nxt_pending = -1;
-      uint32_t nxt_pending_par = 0;
-      uint32_t qr = 0;  // query tiles streamed so far (ring uses)
-      int idx = static_cast<int>(blockIdx.x);
-      bool ok = true;
-      for (int w = 0; ok; ++w) {
-        if (w > 0) {
-          if (!producer_take_item(w, idx, nxt_full, nxt_resp, abort, ctl, kSiteBwdProducer))
-            break;
-          nxt_pending = -1;
-          if (idx < 0) break;
-        }
-        int bh, j, i_start, n_iter;
-        decode(idx, bh, j, i_start, n_iter);
-        if (n_iter > 0) {
-        if (kv_issued > 0 && !mbar_wait(kv_empty, static_cast<uint32_t>(kv_issued - 1) & 1, abort,
-                                        ctl, kSiteBwdProducer))
+    }
+    int last[2] = {-1, -1};
+    int kv_issued = 0;
+    int nxt_pending = -1;
+    uint32_t nxt_pending_par = 0;
+    uint32_t qr = 0;  // query tiles streamed so far (ring uses)
+    int idx = static_cast<int>(blockIdx.x);
+    bool ok = true;
+    for (int w = 0; ok; ++w) {
+      if (w > 0) {
+        if (!producer_take_item(w, idx, nxt_full, nxt_resp, abort, ctl, kSiteBwdProducer)) break;
+        nxt_pending = -1;
+        if (idx < 0) break;
+      }
+      int bh, j, i_start, n_iter;
+      decode(idx, bh, j, i_start, n_iter);
+      if (n_iter > 0) {
+        if (kv_issued > 0 && !wait_all(kv_empty, static_cast<uint32_t>(kv_issued - 1) & 1, abort,
+                                       ctl, kSiteBwdProducer))
           break;
-        mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+        if (leader) {
+          mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
 #pragma unroll
-        for (int b = 0; b < C::NB; ++b) {
-          tma_load_3d(&tm_k, kv_full, smem + C::K_OFF + b * C::BLK, b * 64, j * kT, bh);
-          tma_load_3d(&tm_v, kv_full, smem + C::V_OFF + b * C::BLK, b * 64, j * kT, bh);
+          for (int b = 0; b < C::NB; ++b) {
+            tma_load_3d(&tm_k, kv_full, smem + C::K_OFF + b * C::BLK, b * 64, j * kT, bh);
+            tma_load_3d(&tm_v, kv_full, smem + C::V_OFF + b * C::BLK, b * 64, j * kT, bh);
+          }
         }
+        __syncwarp();
         ++kv_issued;
-        int ic = i_start - 1;  // query tile of the step
+        TileCursor cur(n_t);
         for (int it = 0; it < n_iter; ++it, ++qr) {
-          ic = next_i(ic, j);
+          const int ic = BS ? cur.next(tiles) : i_start + it;  // query tile of the step
           const int st = static_cast<int>(qr & 1);
           const uint32_t u = qr >> 1;
-          if (qr >= 2 && !mbar_wait(qdo_empty + st, (u - 1) & 1, abort, ctl, kSiteBwdProducer)) {
+          if (qr >= 2 && !wait_all(qdo_empty + st, (u - 1) & 1, abort, ctl, kSiteBwdProducer)) {
             ok = false;
             break;
           }
-          const int y = ic * kT;
-          mbar_arrive_expect_tx(q_full + st, C::TILE + 1024);
+          if (leader) {
+            const int y = ic * kT;
+            mbar_arrive_expect_tx(q_full + st, C::TILE + 1024);
 #pragma unroll
-          for (int b = 0; b < C::NB; ++b)
-            tma_load_3d(&tm_q, q_full + st, smem + C::Q_OFF + st * C::TILE + b * C::BLK, b * 64,
-                        y, bh);
-          const size_t vrow = static_cast<size_t>(bh) * Np + y;
-          bulk_load_1d(smem + C::VEC_OFF + st * 1024, lse2 + vrow, 512, q_full + st);
-          bulk_load_1d(smem + C::VEC_OFF + st * 1024 + 512, dvec + vrow, 512, q_full + st);
-          mbar_arrive_expect_tx(do_full + st, C::TILE);
+            for (int b = 0; b < C::NB; ++b)
+              tma_load_3d(&tm_q, q_full + st, smem + C::Q_OFF + st * C::TILE + b * C::BLK,
+                          b * 64, y, bh);
+            const size_t vrow = static_cast<size_t>(bh) * Np + y;
+            bulk_load_1d(smem + C::VEC_OFF + st * 1024, lse2 + vrow, 512, q_full + st);
+            bulk_load_1d(smem + C::VEC_OFF + st * 1024 + 512, dvec + vrow, 512, q_full + st);
+            mbar_arrive_expect_tx(do_full + st, C::TILE);
 #pragma unroll
-          for (int b = 0; b < C::NB; ++b)
-            tma_load_3d(&tm_do, do_full + st, smem + C::DO_OFF + st * C::TILE + b * C::BLK,
-                        b * 64, y, bh);
+            for (int b = 0; b < C::NB; ++b)
+              tma_load_3d(&tm_do, do_full + st, smem + C::DO_OFF + st * C::TILE + b * C::BLK,
+                          b * 64, y, bh);
+          }
+          __syncwarp();
           last[st] = static_cast<int>(u);
         }
         if (!ok) break;
-        }  // n_iter > 0
-        if (!producer_request_item(w, nxt_full, nxt_empty, nxt_resp, abort, ctl,
-                                   kSiteBwdProducer, nxt_pending, nxt_pending_par))
-          break;
       }
-      if (*abort) {
-        if (kv_issued > 0) drain_wait(kv_full, static_cast<uint32_t>(kv_issued - 1) & 1, ctl);
-        for (int s = 0; s < 2; ++s)
-          if (last[s] >= 0) {
-            drain_wait(q_full + s, last[s] & 1, ctl);
-            drain_wait(do_full + s, last[s] & 1, ctl);
-          }
-        if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
-      }
+      if (!producer_request_item(w, nxt_full, nxt_empty, nxt_resp, abort, ctl, kSiteBwdProducer,
+                                 leader, nxt_pending, nxt_pending_par))
+        break;
+    }
+    if (*abort && leader) {
+      if (kv_issued > 0) drain_wait(kv_full, static_cast<uint32_t>(kv_issued - 1) & 1, ctl);
+      for (int s = 0; s < 2; ++s)
+        if (last[s] >= 0) {
+          drain_wait(q_full + s, last[s] & 1, ctl);
+          drain_wait(do_full + s, last[s] & 1, ctl);
+        }
+      if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -546,9 +579,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         continue;
       }
-      int i = i_start - 1;  // query tile of the step
+      TileCursor cur(n_t);
       for (int it = 0; it < n_iter; ++it) {
-        i = next_i(i, j);
+        const int i = BS ? cur.next(tiles) : i_start + it;  // query tile of the step
         const uint32_t g = qbase + it;
         const int st = static_cast<int>(g & 1);
         // LSE2 and D of this half's 64 queries, staged by the producer with
@@ -700,25 +733,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Query tile i and the key tiles it sees for work item idx (group-major,
   // longest query tiles first when causal).
   // With a block mask (BS) only the key tiles whose mask byte (i, j) is set
-  // are visited; next_j steps to the next of them.
-  const uint8_t* hrow = nullptr;  // this item's mask row (BS)
+  // are visited (`tiles`, walked with a TileCursor).  Every role calls this
+  // with its whole (converged) warp.
+  RowTiles tiles{bmask, n_t, 0};
   auto decode = [&](int idx, int& bh, int& i, int& n_kv) {
     int t;
     group_major(idx, n_t, BH, group, bh, t);
     i = n_t - 1 - t;
     n_kv = CAUSAL ? i + 1 : n_t;
     if (BS) {
-      hrow = bmask + (static_cast<size_t>(mask_heads == 1 ? 0 : bh % H) * n_t + i) * n_t;
-      const int jend = n_kv;
-      n_kv = 0;
-      for (int j = 0; j < jend; ++j) n_kv += hrow[j] != 0;
+      tiles = RowTiles{bmask + (static_cast<size_t>(mask_heads == 1 ? 0 : bh % H) * n_t + i) * n_t,
+                       n_t, n_kv};
+      n_kv = count_tiles(tiles);
     }
-  };
-  auto next_j = [&](int j) -> int {
-    ++j;
-    if (BS)
-      while (j < n_t && hrow[j] == 0) ++j;
-    return j;
   };
 
   if (threadIdx.x == 0) {
@@ -757,84 +784,93 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the loop (it reads the block mask with all lanes);
+    // the elected lane issues the copies and the next-item requests.
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      int last_k[C::NK], last_v[C::NV];
+    }
+    int last_k[C::NK], last_v[C::NV];
 #pragma unroll
-      for (int s = 0; s < C::NK; ++s) last_k[s] = -1;
+    for (int s = 0; s < C::NK; ++s) last_k[s] = -1;
 #pragma unroll
-      for (int s = 0; s < C::NV; ++s) last_v[s] = -1;
-      int q_issued = 0;
-      int nxt_pending = -1;
-      uint32_t nxt_pending_par = 0;
-      uint32_t kr = 0;  // key tiles streamed so far (ring uses of both rings)
-      int idx = static_cast<int>(blockIdx.x);
-      bool ok = true;
-      for (int it = 0; ok; ++it) {
-        if (it > 0) {
-          if (!producer_take_item(it, idx, nxt_full, nxt_resp, abort, ctl, kSiteBwdProducer))
-            break;
-          nxt_pending = -1;
-          if (idx < 0) break;
-        }
-        int bh, i, n_kv;
-        decode(idx, bh, i, n_kv);
-        if (n_kv > 0) {
-        if (q_issued > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(q_issued - 1) & 1, abort,
-                                       ctl, kSiteBwdProducer))
+    for (int s = 0; s < C::NV; ++s) last_v[s] = -1;
+    int q_issued = 0;
+    int nxt_pending = -1;
+    uint32_t nxt_pending_par = 0;
+    uint32_t kr = 0;  // key tiles streamed so far (ring uses of both rings)
+    int idx = static_cast<int>(blockIdx.x);
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      if (it > 0) {
+        if (!producer_take_item(it, idx, nxt_full, nxt_resp, abort, ctl, kSiteBwdProducer)) break;
+        nxt_pending = -1;
+        if (idx < 0) break;
+      }
+      int bh, i, n_kv;
+      decode(idx, bh, i, n_kv);
+      if (n_kv > 0) {
+        if (q_issued > 0 && !wait_all(q_empty, static_cast<uint32_t>(q_issued - 1) & 1, abort,
+                                      ctl, kSiteBwdProducer))
           break;
-        mbar_arrive_expect_tx(q_full, 2 * C::TILE);
+        if (leader) {
+          mbar_arrive_expect_tx(q_full, 2 * C::TILE);
 #pragma unroll
-        for (int b = 0; b < C::NB; ++b) {
-          tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + b * C::BLK, b * 64, i * kT, bh);
-          tma_load_3d(&tm_do, q_full, smem + C::DO_OFF + b * C::BLK, b * 64, i * kT, bh);
+          for (int b = 0; b < C::NB; ++b) {
+            tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + b * C::BLK, b * 64, i * kT, bh);
+            tma_load_3d(&tm_do, q_full, smem + C::DO_OFF + b * C::BLK, b * 64, i * kT, bh);
+          }
         }
+        __syncwarp();
         ++q_issued;
-        int jt = -1;  // key tile of the step
+        TileCursor cur(n_t);
         for (int jj = 0; jj < n_kv; ++jj, ++kr) {
-          jt = next_j(jt);
+          const int jt = BS ? cur.next(tiles) : jj;  // key tile of the step
           const int sk = static_cast<int>(kr % C::NK), sv = static_cast<int>(kr % C::NV);
           const uint32_t uk = kr / C::NK, uv = kr / C::NV;
-          if (kr >= C::NK &&
-              !mbar_wait(k_empty + sk, (uk - 1) & 1, abort, ctl, kSiteBwdProducer)) {
+          if (kr >= C::NK && !wait_all(k_empty + sk, (uk - 1) & 1, abort, ctl, kSiteBwdProducer)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(k_full + sk, C::TILE);
+          if (leader) {
+            mbar_arrive_expect_tx(k_full + sk, C::TILE);
 #pragma unroll
-          for (int b = 0; b < C::NB; ++b)
-            tma_load_3d(&tm_k, k_full + sk, smem + C::K_OFF + sk * C::TILE + b * C::BLK, b * 64,
-                        jt * kT, bh);
+            for (int b = 0; b < C::NB; ++b)
+              tma_load_3d(&tm_k, k_full + sk, smem + C::K_OFF + sk * C::TILE + b * C::BLK, b * 64,
+                          jt * kT, bh);
+          }
+          __syncwarp();
           last_k[sk] = static_cast<int>(uk);
-          if (kr >= C::NV &&
-              !mbar_wait(v_empty + sv, (uv - 1) & 1, abort, ctl, kSiteBwdProducer)) {
+          if (kr >= C::NV && !wait_all(v_empty + sv, (uv - 1) & 1, abort, ctl, kSiteBwdProducer)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(v_full + sv, C::TILE);
+          if (leader) {
+            mbar_arrive_expect_tx(v_full + sv, C::TILE);
 #pragma unroll
-          for (int b = 0; b < C::NB; ++b)
-            tma_load_3d(&tm_v, v_full + sv, smem + C::V_OFF + sv * C::TILE + b * C::BLK, b * 64,
-                        jt * kT, bh);
+            for (int b = 0; b < C::NB; ++b)
+              tma_load_3d(&tm_v, v_full + sv, smem + C::V_OFF + sv * C::TILE + b * C::BLK, b * 64,
+                          jt * kT, bh);
+          }
+          __syncwarp();
           last_v[sv] = static_cast<int>(uv);
         }
         if (!ok) break;
-        }  // n_kv > 0
-        if (!producer_request_item(it, nxt_full, nxt_empty, nxt_resp, abort, ctl,
-                                   kSiteBwdProducer, nxt_pending, nxt_pending_par))
-          break;
       }
-      if (*abort) {
-        if (q_issued > 0) drain_wait(q_full, static_cast<uint32_t>(q_issued - 1) & 1, ctl);
-        for (int s = 0; s < C::NK; ++s)
-          if (last_k[s] >= 0) drain_wait(k_full + s, last_k[s] & 1, ctl);
-        for (int s = 0; s < C::NV; ++s)
-          if (last_v[s] >= 0) drain_wait(v_full + s, last_v[s] & 1, ctl);
-        if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
-      }
+      if (!producer_request_item(it, nxt_full, nxt_empty, nxt_resp, abort, ctl, kSiteBwdProducer,
+                                 leader, nxt_pending, nxt_pending_par))
+        break;
+    }
+    if (*abort && leader) {
+      if (q_issued > 0) drain_wait(q_full, static_cast<uint32_t>(q_issued - 1) & 1, ctl);
+      for (int s = 0; s < C::NK; ++s)
+        if (last_k[s] >= 0) drain_wait(k_full + s, last_k[s] & 1, ctl);
+      for (int s = 0; s < C::NV; ++s)
+        if (last_v[s] >= 0) drain_wait(v_full + s, last_v[s] & 1, ctl);
+      if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -982,9 +1018,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float my_l2 = lse2[static_cast<size_t>(bh) * Np + q_idx];  // +inf past N
       const float my_d = dvec[static_cast<size_t>(bh) * Np + q_idx];
-      int jt = -1;  // key tile of the step
+      TileCursor cur(n_t);
       for (int jj = 0; jj < n_kv; ++jj) {
-        jt = next_j(jt);
+        const int jt = BS ? cur.next(tiles) : jj;  // key tile of the step
         const uint32_t g = kbase + jj;
         const uint32_t col_s = kQColS + (g & 1) * kT + 64 * h;
         if (!wait_all(s_full + (g & 1), (g >> 1) & 1, abort, ctl, kSiteBwdSoftmax)) {

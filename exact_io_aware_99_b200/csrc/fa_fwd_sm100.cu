@@ -40,6 +40,8 @@
 // time, so their K and V stay in L2), longest-first inside a group.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -50,10 +52,17 @@ constexpr int kBM = 128;              // query rows per tile (TMEM lanes)
 constexpr int kBN = 128;              // keys per K/V tile
 constexpr int kThreads = 384;         // 2 softmax warpgroups + producer/MMA warpgroup
 // Registers per thread: 168 at launch (384 threads), then the softmax
-// warpgroups take 224 and the producer/MMA warpgroup keeps 56:
-// 224 + 224 + 56 = 504 = 3 x 168, the launch budget of each lane slot.
-constexpr int kLaunchRegs = 168, kSoftmaxRegs = 224, kControlRegs = 56;
-static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kLaunchRegs, "register split over budget");
+// warpgroups take RegSplit::kSoftmax each and the producer/MMA warpgroup keeps the
+// rest: 224 + 224 + 56 = 504 = 3 x 168, the launch budget of each lane slot.
+// With a block mask the producer walks the mask with its whole warp and
+// needs more, so the split is 216 + 216 + 72.
+constexpr int kLaunchRegs = 168;
+template <bool BS>
+struct RegSplit {
+  static constexpr int kSoftmax = BS ? 216 : 224;
+  static constexpr int kControl = 3 * kLaunchRegs - 2 * kSoftmax;
+  static_assert(2 * kSoftmax + kControl <= 3 * kLaunchRegs, "register split over budget");
+};
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 #ifndef FA_FWD_POLY_EVERY
 #define FA_FWD_POLY_EVERY 0  // one column pair in this many uses the FMA-pipe exp2 (0: none)
@@ -135,14 +144,14 @@ struct ItemTiles {
     return has[x] && (!CAUSAL || j <= qt[x]) && row[x][j] != 0;
   }
   __device__ __forceinline__ bool any(int j) const { return active(0, j) || active(1, j); }
-  // First visited key tile after j (n_t when there is none).
-  __device__ __forceinline__ int next(int j) const {
-    do {
-      ++j;
-    } while (j < n_t && !any(j));
-    return j;
+  // Bit b of word w: key tile 32 w + b is visited.  Called by all 32 lanes
+  // of a converged warp (each lane reads one tile's mask bytes).
+  __device__ __forceinline__ uint32_t word(int w) const {
+    const int j = 32 * w + lane_id();
+    return __ballot_sync(0xffffffffu, j < n_t && any(j));
   }
 };
+
 
 // Steps of a work item and, with a block mask, the tiles it visits.  Dense:
 // tile x visits key tiles [0, n_x[x]); block-sparse: both tiles step through
@@ -162,7 +171,7 @@ __device__ __forceinline__ void item_plan(int idx, int n_t, int BH, int group, i
     }
     it.n_t = n_t;
     int steps = 0;
-    for (int j = it.next(-1); j < n_t; j = it.next(j)) ++steps;
+    for (int w = 0; w < (n_t + 31) / 32; ++w) steps += __popc(it.word(w));
     n_x[0] = steps;
     n_x[1] = it.has[1] ? steps : 0;
   }
@@ -251,17 +260,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp >= 8) {
-  regs_decrease<kControlRegs>();
+  regs_decrease<RegSplit<BS>::kControl>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+    // Dense launches run the producer on one lane.  With a block mask the
+    // whole warp runs the loop (it reads the mask with all lanes, see
+    // ItemTiles::word) and the elected lane issues the copies and requests.
+    auto produce = [&](auto warp_mode) {
+      constexpr bool W = decltype(warp_mode)::value;
+      const bool leader = W ? elect_one() : true;
+      auto wait = [&](uint64_t* bar, uint32_t par) -> bool {
+        return W ? wait_all(bar, par, abort, ctl, kSiteFwdProducer)
+                 : mbar_wait(bar, par, abort, ctl, kSiteFwdProducer);
+      };
+      auto sync = [&]() {
+        if (W) __syncwarp();
+      };
+      if (leader) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+      }
       int last_k[C::NST], last_v[C::NST];
 #pragma unroll
       for (int s = 0; s < C::NST; ++s) last_k[s] = last_v[s] = -1;
-      int q_issued = 0;           // Q loads issued (one per item)
+      int q_issued = 0;           // Q loads issued (one per item with work)
       int nxt_pending = -1;       // slot of a request in flight
       uint32_t nxt_pending_par = 0;
       uint32_t kv = 0;            // K/V ring uses so far
@@ -270,9 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok; ++i) {
         if (i > 0) {
           const int sl = i & 1;
-          if (!mbar_wait(nxt_full + sl, static_cast<uint32_t>((i - 1) >> 1) & 1, abort, ctl,
-                         kSiteFwdProducer))
-            break;
+          if (!wait(nxt_full + sl, static_cast<uint32_t>((i - 1) >> 1) & 1)) break;
           nxt_pending = -1;
           idx = clc_result_x(nxt_resp + 16 * sl);
           if (idx < 0) break;
@@ -282,57 +303,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
         const int n_max = max(n_x[0], n_x[1]);
         if (n_max > 0) {
-        // Q of this item replaces the previous item's once its S MMAs are done.
-        if (q_issued > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(q_issued - 1) & 1, abort,
-                                       ctl, kSiteFwdProducer))
-          break;
-        const int nq = n_x[1] > 0 ? 2 : 1;
-        mbar_arrive_expect_tx(q_full, nq * C::TILE);
-        for (int x = 0; x < nq; ++x)
+          // Q of this item replaces the previous item's once its S MMAs are done.
+          if (q_issued > 0 && !wait(q_empty, static_cast<uint32_t>(q_issued - 1) & 1)) break;
+          if (leader) {
+            const int nq = n_x[1] > 0 ? 2 : 1;
+            mbar_arrive_expect_tx(q_full, nq * C::TILE);
+            for (int x = 0; x < nq; ++x)
 #pragma unroll
-          for (int b = 0; b < C::NB; ++b)
-            tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + x * C::TILE + b * C::BLK, b * 64,
-                        (2 * pair + x) * kBM, bh);
-        ++q_issued;
-        int jt = -1;  // key tile of the step
-        for (int j = 0; j < n_max; ++j, ++kv) {
-          jt = BS ? tiles.next(jt) : j;
-          const int s = static_cast<int>(kv % C::NST);
-          const uint32_t u = kv / C::NST;
-          if (kv >= C::NST && !mbar_wait(k_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer)) {
-            ok = false;
-            break;
+              for (int b = 0; b < C::NB; ++b)
+                tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + x * C::TILE + b * C::BLK, b * 64,
+                            (2 * pair + x) * kBM, bh);
           }
-          mbar_arrive_expect_tx(k_full + s, C::TILE);
+          sync();
+          ++q_issued;
+          TileCursor cur(n_t);
+          for (int j = 0; j < n_max; ++j, ++kv) {
+            const int jt = BS ? cur.next(tiles) : j;  // key tile of the step
+            const int s = static_cast<int>(kv % C::NST);
+            const uint32_t u = kv / C::NST;
+            if (kv >= C::NST && !wait(k_empty + s, (u - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            if (leader) {
+              mbar_arrive_expect_tx(k_full + s, C::TILE);
 #pragma unroll
-          for (int b = 0; b < C::NB; ++b)
-            tma_load_3d(&tm_k, k_full + s, smem + C::K_OFF + s * C::TILE + b * C::BLK, b * 64,
-                        jt * kBN, bh);
-          last_k[s] = static_cast<int>(u);
-          if (kv >= C::NST && !mbar_wait(v_empty + s, (u - 1) & 1, abort, ctl, kSiteFwdProducer)) {
-            ok = false;
-            break;
+              for (int b = 0; b < C::NB; ++b)
+                tma_load_3d(&tm_k, k_full + s, smem + C::K_OFF + s * C::TILE + b * C::BLK,
+                            b * 64, jt * kBN, bh);
+            }
+            sync();
+            last_k[s] = static_cast<int>(u);
+            if (kv >= C::NST && !wait(v_empty + s, (u - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            if (leader) {
+              mbar_arrive_expect_tx(v_full + s, C::TILE);
+#pragma unroll
+              for (int b = 0; b < C::NB; ++b)
+                tma_load_3d(&tm_v, v_full + s, smem + C::V_OFF + s * C::TILE + b * C::BLK,
+                            b * 64, jt * kBN, bh);
+            }
+            sync();
+            last_v[s] = static_cast<int>(u);
           }
-          mbar_arrive_expect_tx(v_full + s, C::TILE);
-#pragma unroll
-          for (int b = 0; b < C::NB; ++b)
-            tma_load_3d(&tm_v, v_full + s, smem + C::V_OFF + s * C::TILE + b * C::BLK, b * 64,
-                        jt * kBN, bh);
-          last_v[s] = static_cast<int>(u);
+          if (!ok) break;
         }
-        if (!ok) break;
-        }  // n_max > 0
         // Ask for the next item now, while this one's MMAs and softmax run.
         const int sl1 = (i + 1) & 1;
         const uint32_t u1 = static_cast<uint32_t>(i >> 1);
-        if (u1 > 0 && !mbar_wait(nxt_empty + sl1, (u1 - 1) & 1, abort, ctl, kSiteFwdProducer))
-          break;
-        mbar_arrive_expect_tx(nxt_full + sl1, 16);
-        clc_try_cancel(nxt_resp + 16 * sl1, nxt_full + sl1);
+        if (u1 > 0 && !wait(nxt_empty + sl1, (u1 - 1) & 1)) break;
+        if (leader) {
+          mbar_arrive_expect_tx(nxt_full + sl1, 16);
+          clc_try_cancel(nxt_resp + 16 * sl1, nxt_full + sl1);
+        }
+        sync();
         nxt_pending = sl1;
         nxt_pending_par = u1 & 1;
       }
-      if (*abort) {
+      if (*abort && leader) {
         // Let every copy and request this CTA started land before shared
         // memory is released.
         if (q_issued > 0) drain_wait(q_full, static_cast<uint32_t>(q_issued - 1) & 1, ctl);
@@ -342,7 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
       }
-    }
+    };
+    if (BS)
+      produce(std::true_type{});
+    else if (lane == 0)
+      produce(std::false_type{});
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
@@ -449,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
   } else {
-    regs_increase<kSoftmaxRegs>();
+    regs_increase<RegSplit<BS>::kSoftmax>();
     // --------------------------------------- softmax (warps 0-3: A, 4-7: B)
     const int x = warp >> 2;
     const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
@@ -481,9 +515,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float m = -INFINITY;  // reference max, base-2 scaled units
       float l = 0.f;
-      int jt = -1;          // key tile of the step
+      TileCursor cur(n_t);
       for (int j = 0; j < n_kv; ++j) {
-        jt = BS ? tiles.next(jt) : j;
+        const int jt = BS ? cur.next(tiles) : j;  // key tile of the step
         if (!wait_all(s_full + x, (s_base + j) & 1, abort, ctl, kSiteFwdSoftmax)) {
           ok = false;
           break;

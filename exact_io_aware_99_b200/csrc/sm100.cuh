@@ -159,29 +159,37 @@ __device__ __forceinline__ bool next_work_item(int it, int& idx, uint64_t* full,
   return true;
 }
 
-// Producer side (one thread): the answer for item it >= 1.
+// Producer side, called by all lanes of the producer warp: the answer for
+// item it >= 1.
 __device__ __forceinline__ bool producer_take_item(int it, int& idx, uint64_t* full,
                                                    const uint8_t* resp, volatile int* abort,
                                                    const WaitCtl& ctl, int site) {
   const int sl = it & 1;
-  if (!mbar_wait(full + sl, static_cast<uint32_t>((it - 1) >> 1) & 1, abort, ctl, site))
-    return false;
+  const bool w = mbar_wait(full + sl, static_cast<uint32_t>((it - 1) >> 1) & 1, abort, ctl, site);
+  if (!__all_sync(0xffffffffu, w)) return false;
   idx = clc_result_x(resp + 16 * sl);
   return true;
 }
 
-// Producer side (one thread): request item it + 1 into slot (it + 1) & 1
-// once the consumers have read that slot's previous answer.  `pending` and
+// Producer side, called by all lanes of the producer warp: request item
+// it + 1 into slot (it + 1) & 1 once the consumers have read that slot's
+// previous answer; `leader` (one lane) issues it.  `pending` and
 // `pending_par` record the request in flight (drained on abort).
 __device__ __forceinline__ bool producer_request_item(int it, uint64_t* full, uint64_t* empty,
                                                       uint8_t* resp, volatile int* abort,
-                                                      const WaitCtl& ctl, int site, int& pending,
-                                                      uint32_t& pending_par) {
+                                                      const WaitCtl& ctl, int site, bool leader,
+                                                      int& pending, uint32_t& pending_par) {
   const int sl = (it + 1) & 1;
   const uint32_t u = static_cast<uint32_t>(it >> 1);
-  if (u > 0 && !mbar_wait(empty + sl, (u - 1) & 1, abort, ctl, site)) return false;
-  mbar_arrive_expect_tx(full + sl, 16);
-  clc_try_cancel(resp + 16 * sl, full + sl);
+  if (u > 0) {
+    const bool w = mbar_wait(empty + sl, (u - 1) & 1, abort, ctl, site);
+    if (!__all_sync(0xffffffffu, w)) return false;
+  }
+  if (leader) {
+    mbar_arrive_expect_tx(full + sl, 16);
+    clc_try_cancel(resp + 16 * sl, full + sl);
+  }
+  __syncwarp();
   pending = sl;
   pending_par = u & 1;
   return true;
@@ -438,6 +446,26 @@ __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v &
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+// Walks a set of tiles in increasing order, 32 tiles per word: `t.word(w)`
+// returns the bits of tiles 32 w .. 32 w + 31 (computed by a converged warp,
+// e.g. with a ballot), `t.n_t` the number of tiles.  Warp-uniform: every lane
+// holds the same state.
+struct TileCursor {
+  int w = -1, nw;
+  uint32_t bits = 0;
+  __device__ explicit TileCursor(int n_t) : nw((n_t + 31) / 32) {}
+  template <class Tiles>
+  __device__ __forceinline__ int next(const Tiles& t) {
+    while (bits == 0) {
+      if (++w >= nw) return t.n_t;
+      bits = t.word(w);
+    }
+    const int b = __ffs(bits) - 1;
+    bits &= bits - 1;
+    return 32 * w + b;
+  }
+};
 
 // One lane of a converged warp (elect.sync over the full mask).  The MMA
 // issuers run their whole loop on all 32 lanes -- waits, fences and branches

@@ -27,3 +27,44 @@ def fwd_bytes(B: int, H: int, N: int, d: int, elem: int = 2) -> float:
 
 def bwd_bytes(B: int, H: int, N: int, d: int, elem: int = 2) -> float:
     return 8.0 * B * H * N * d * elem + 4.0 * B * H * N
+
+
+def visible_pairs(block_mask, N: int, causal: bool, block: int = 128) -> float:
+    """Number of (query, key) pairs a block mask (bool [Hm, nt, nt] or
+    [nt, nt]) leaves visible, summed over its heads, with ragged edge tiles
+    and the causal triangle counted exactly."""
+    import numpy as np
+    m = np.asarray(block_mask, dtype=bool)
+    if m.ndim == 2:
+        m = m[None]
+    nt = m.shape[-1]
+    size = np.full(nt, block, dtype=np.float64)
+    size[-1] = N - block * (nt - 1)
+    total = 0.0
+    for i in range(nt):
+        for j in range(nt):
+            if causal and j > i:
+                continue
+            if causal and j == i:
+                s = size[i]
+                pairs = s * (s + 1) / 2
+            else:
+                pairs = size[i] * size[j]
+            total += pairs * float(np.count_nonzero(m[:, i, j]))
+    return total
+
+
+def fwd_flops_masked(B: int, H: int, N: int, d: int, causal: bool, block_mask) -> float:
+    """Forward FLOPs of block-sparse attention: 4 d per visible (query, key)
+    pair (the dense count with only the visible pairs).  A per-head mask
+    (H heads) is counted per head; a shared mask is counted H times."""
+    import numpy as np
+    m = np.asarray(block_mask, dtype=bool)
+    heads = 1 if m.ndim == 2 else m.shape[0]
+    pairs = visible_pairs(m, N, causal)
+    per_batch = pairs * (H if heads == 1 else 1)
+    return 4.0 * d * B * per_batch
+
+
+def bwd_flops_masked(B: int, H: int, N: int, d: int, causal: bool, block_mask) -> float:
+    return 2.5 * fwd_flops_masked(B, H, N, d, causal, block_mask)

@@ -139,3 +139,24 @@ def test_inputs_are_seeded_and_rounded():
     big = workloads.make_inputs(workloads.WORKLOADS["gpt3_d80"], B=1, H=32, N=64)
     var = big["k"].float().var().item()
     assert 0.85 < var < 1.2
+
+
+def test_masked_flop_counts_reduce_to_the_dense_ones():
+    import numpy as np
+    from exact_io_aware_99_b200 import perf
+    for N in (1, 127, 128, 300, 1000):
+        nt = (N + 127) // 128
+        ones = np.ones((nt, nt), bool)
+        for causal in (False, True):
+            dense = N * (N + 1) / 2 if causal else float(N * N)
+            assert perf.visible_pairs(ones, N, causal) == dense
+        # masked flops of an all-ones mask = the dense count (H heads shared)
+        assert perf.fwd_flops_masked(2, 3, N, 64, False, ones) == perf.fwd_flops(2, 3, N, 64, False)
+    # one visible interior block of a 3 x 3 mask: 128 x 128 pairs
+    m = np.zeros((3, 3), bool)
+    m[1, 0] = True
+    assert perf.visible_pairs(m, 300, False) == 128 * 128
+    # per-head masks are counted per head
+    mh = np.zeros((2, 3, 3), bool)
+    mh[0, 1, 0] = mh[1, 2, 2] = True           # tile 2 is 44 rows: 44 x 44
+    assert perf.fwd_flops_masked(1, 2, 300, 8, False, mh) == 4 * 8 * (128 * 128 + 44 * 44)

@@ -11,6 +11,11 @@ Workloads (shapes are [B, H, N, d], d fastest):
 * ``fwd_d64``     B8 H16 N1024 d64, bf16, forward only, non-causal.
 * ``causal_d128`` B4 H16 N4096 d128, bf16, causal, forward+backward.
 * ``long_d128``   B1 H16 N16384 d128, bf16, causal, forward+backward.
+* ``bsparse_d128`` B1 H16 N16384 d128, bf16, non-causal, forward+backward,
+  block-sparse: every query tile sees the key tiles within 4 tiles of its
+  own plus key tiles 0 and 1 (a local window with global tokens, the hybrid
+  local + global pattern the FlashAttention-2 review names for sparse
+  attention); 128 x 128 tiles, one mask for all heads, ~8.6 % of the pairs.
 * ``gpt3_d80``    B8 H32 N2048 d80, bf16, causal, forward+backward; Q, K, V
   are projections X.W of a unit-normal activation X [B, N, 2560] through
   three independent N(0, 0.02^2) [2560, 2560] weights, then split into
@@ -43,6 +48,7 @@ class Workload:
     backward: bool
     projected: bool = False   # Q/K/V = X.W (GPT-3 shaped layer)
     hidden: int = 0
+    mask: str = ""            # block-sparse pattern name ("" = dense)
 
     @property
     def scale(self) -> float:
@@ -59,8 +65,9 @@ class Workload:
     def describe(self) -> str:
         pas = "fwd+bwd" if self.backward else "fwd"
         cz = "causal" if self.causal else "non-causal"
+        bs = f" block-sparse {self.mask}" if self.mask else ""
         return (f"{self.name}: B{self.B} H{self.H} N{self.N} d{self.d} "
-                f"{self.dtype} {cz} {pas}")
+                f"{self.dtype} {cz}{bs} {pas}")
 
 
 WORKLOADS: Dict[str, Workload] = {
@@ -71,8 +78,27 @@ WORKLOADS: Dict[str, Workload] = {
         Workload("long_d128", 3, 1, 16, 16384, 128, "bf16", True, True),
         Workload("gpt3_d80", 4, 8, 32, 2048, 80, "bf16", True, True,
                  projected=True, hidden=2560),
+        Workload("bsparse_d128", 5, 1, 16, 16384, 128, "bf16", False, True,
+                 mask="local4_global2"),
     ]
 }
+
+
+def block_mask(w: Workload, N: Optional[int] = None):
+    """The workload's block mask as numpy bool [1, nt, nt] (128-row tiles),
+    or None for a dense workload.  ``local4_global2``: query tile I sees key
+    tiles J with |I - J| <= 4, and key tiles 0 and 1."""
+    import numpy as np
+    if not w.mask:
+        return None
+    N = w.N if N is None else N
+    nt = (N + 127) // 128
+    if w.mask == "local4_global2":
+        i = np.arange(nt)
+        m = np.abs(i[:, None] - i[None, :]) <= 4
+        m[:, :2] = True
+        return m[None]
+    raise ValueError(f"unknown mask pattern {w.mask}")
 
 
 def round_to(x: torch.Tensor, dtype: torch.dtype) -> torch.Tensor:
