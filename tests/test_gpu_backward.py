@@ -37,16 +37,16 @@ def test_bf16_backward_several_heads():
     check_backward(x["q"], x["k"], x["v"], x["do"], 1 / math.sqrt(128), True)
 
 
-def test_bf16_backward_is_repeatable_within_tolerance():
-    # dQ is summed with atomics, so bits may differ between runs, but both
-    # runs must meet the oracle bound (checked inside) and agree closely.
+def test_bf16_backward_is_bitwise_reproducible():
+    # Every gradient tile is accumulated by one CTA in a fixed order (no
+    # atomics), whichever CTA ends up running it: two runs agree bit for bit.
     from gpu_cases import gpu_backward, gpu_forward
     x = workloads.random_case(1, 4, 1024, 64, 7)
     o, lse = gpu_forward(x["q"], x["k"], x["v"], 0.125, True)
     a = gpu_backward(x["q"], x["k"], x["v"], o, x["do"], lse, 0.125, True)
     b = gpu_backward(x["q"], x["k"], x["v"], o, x["do"], lse, 0.125, True)
     for ga, gb in zip(a, b):
-        assert float((ga.float() - gb.float()).abs().max()) <= 1e-2 * float(ga.float().abs().max())
+        assert torch.equal(ga, gb)
 
 
 def _sample_heads(B, H, n, seed):
