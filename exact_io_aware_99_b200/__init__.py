@@ -7,6 +7,7 @@ used for device memory and streams.
 Low-level entry points (same names as the C ABI): ``fa_forward``,
 ``fa_forward_ex``, ``fa_backward``, ``fa_backward_ex``,
 ``fa_backward_noalloc``, ``fa_forward_blocksparse``, ``fa_backward_blocksparse``,
+``fa_forward_splitkv``, ``fa_splitkv_default_splits``, ``fa_splitkv_workspace_size``,
 ``fa_backward_workspace_size``,
 ``fa_status_string``, ``fa_device_status``, ``fa_set_wait_timeout_ns``,
 ``fa_selftest_wait_timeout``.
@@ -14,7 +15,9 @@ Low-level entry points (same names as the C ABI): ``fa_forward``,
 Convenience wrappers that allocate outputs with torch:
 ``attention_forward(q, k, v, scale=None, causal=False, block_mask=None)
 -> (o, lse)`` and ``attention_backward(q, k, v, o, do, lse, scale=None,
-causal=False, block_mask=None) -> (dq, dk, dv)``.
+causal=False, block_mask=None) -> (dq, dk, dv)``, and
+``attention_decode(q, k, v, scale=None, causal=False, num_splits=None)
+-> (o, lse)`` for N_q queries against N_k keys (split-KV).
 
 The shared library is loaded on first use of any of these names (so the
 ``build`` submodule can run before it exists); using them without the built
@@ -27,9 +30,10 @@ _NATIVE = {
     "fa_forward_ex", "fa_backward", "fa_backward_ex", "fa_backward_noalloc",
     "fa_backward_workspace_size", "fa_status_string", "fa_device_status",
     "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_forward_blocksparse",
-    "fa_backward_blocksparse",
+    "fa_backward_blocksparse", "fa_forward_splitkv", "fa_splitkv_default_splits",
+    "fa_splitkv_workspace_size",
 }
-_API = {"attention_forward", "attention_backward"}
+_API = {"attention_forward", "attention_backward", "attention_decode"}
 
 
 def __getattr__(name):

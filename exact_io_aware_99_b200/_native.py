@@ -30,7 +30,8 @@ EXPORTS = (
     "fa_forward", "fa_forward_ex", "fa_backward_workspace_size", "fa_backward",
     "fa_backward_ex", "fa_status_string", "fa_last_cuda_error", "fa_device_status",
     "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_backward_noalloc",
-    "fa_forward_blocksparse", "fa_backward_blocksparse",
+    "fa_forward_blocksparse", "fa_backward_blocksparse", "fa_forward_splitkv",
+    "fa_splitkv_default_splits", "fa_splitkv_workspace_size",
 )
 
 # Size of the library's built-in scratch array used by fa_backward_noalloc.
@@ -78,6 +79,12 @@ def _load() -> ctypes.CDLL:
     lib.fa_backward_blocksparse.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I,
                                             P, S, P]
     lib.fa_backward_blocksparse.restype = I
+    lib.fa_forward_splitkv.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, P, S, P]
+    lib.fa_forward_splitkv.restype = I
+    lib.fa_splitkv_default_splits.argtypes = [I, I, I, I]
+    lib.fa_splitkv_default_splits.restype = I
+    lib.fa_splitkv_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.fa_splitkv_workspace_size.restype = S
     lib.fa_backward_noalloc.restype = I
     return lib
 
@@ -198,3 +205,19 @@ def fa_backward_blocksparse(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, 
                                       int(bool(causal)), _ptr(block_mask), int(mask_heads),
                                       _ptr(workspace), int(workspace_bytes), _stream(stream))
     return _check(st, "fa_backward_blocksparse", check)
+
+
+def fa_forward_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, num_splits, workspace,
+                       workspace_bytes, stream=None, check=True) -> int:
+    st = _lib.fa_forward_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                                 float(scale), int(bool(causal)), int(num_splits),
+                                 _ptr(workspace), int(workspace_bytes), _stream(stream))
+    return _check(st, "fa_forward_splitkv", check)
+
+
+def fa_splitkv_default_splits(B, H, Nq, Nk) -> int:
+    return int(_lib.fa_splitkv_default_splits(B, H, Nq, Nk))
+
+
+def fa_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits) -> int:
+    return int(_lib.fa_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits))

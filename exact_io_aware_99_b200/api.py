@@ -87,3 +87,25 @@ def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
         nat.fa_backward_ex(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, scale, causal,
                            workspace, wbytes, _dtype_code(q))
     return dq, dk, dv
+
+
+def attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                     scale: Optional[float] = None, causal: bool = False,
+                     num_splits: Optional[int] = None
+                     ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split-KV forward (bf16): q [B, H, N_q, d] against k, v [B, H, N_k, d];
+    see ``fa_forward_splitkv``.  Returns O [B, H, N_q, d] and LSE [B, H, N_q]."""
+    _check_inputs(k, v)
+    if not q.is_cuda or not q.is_contiguous() or q.dtype != k.dtype or q.dim() != 4 \
+            or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
+        raise ValueError("q must be a contiguous CUDA [B, H, N_q, d] tensor matching k and v")
+    B, H, Nq, d = _dims(q)
+    Nk = int(k.shape[2])
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    s = nat.fa_splitkv_default_splits(B, H, Nq, Nk) if num_splits is None else int(num_splits)
+    wbytes = nat.fa_splitkv_workspace_size(B, H, Nq, Nk, d, s)
+    ws = torch.empty(wbytes, device=q.device, dtype=torch.uint8)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32)
+    nat.fa_forward_splitkv(q, k, v, out, lse, B, H, Nq, Nk, d, scale, causal, s, ws, wbytes)
+    return out, lse

@@ -341,6 +341,81 @@ fa_status fa_backward_blocksparse(const void* q, const void* k, const void* v, c
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
+// Split-KV partition: the N_k keys' tiles split into ranges of kt_per tiles
+// (the last range may be shorter; none is empty).
+struct SplitPlan {
+  int n_split, kt_per;
+};
+SplitPlan split_plan(int Nk, int num_splits) {
+  const int n_kt = (Nk + 127) / 128;
+  int s = num_splits < 1 ? 1 : (num_splits > n_kt ? n_kt : num_splits);
+  const int kt_per = (n_kt + s - 1) / s;
+  s = (n_kt + kt_per - 1) / kt_per;
+  return {s, kt_per};
+}
+
+struct SplitWs {
+  size_t lse_off, total;
+};
+SplitWs splitkv_ws(int B, int H, int Nq, int d, int n_split) {
+  const size_t rows = static_cast<size_t>(n_split) * B * H * Nq;
+  const size_t o_bytes = up256(rows * d * sizeof(float));
+  return {o_bytes, o_bytes + up256(rows * sizeof(float))};
+}
+
+int fa_splitkv_default_splits(int B, int H, int Nq, int Nk) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return 0;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long items = static_cast<long long>(B) * H * (((Nq + 127) / 128 + 1) / 2);
+  const long long want = (2LL * sms + items - 1) / items;  // about two items per SM
+  const int n_kt = (Nk + 127) / 128;
+  const int s = static_cast<int>(want < 1 ? 1 : (want > n_kt ? n_kt : want));
+  return split_plan(Nk, s).n_split;
+}
+
+size_t fa_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || d < 1 || d > 128 || num_splits < 1) return 0;
+  return splitkv_ws(B, H, Nq, d, split_plan(Nk, num_splits).n_split).total;
+}
+
+fa_status fa_forward_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                             int num_splits, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (!q || !k || !v || !o || !lse || num_splits < 1) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, Nq, d, scale, FA_BF16);
+  if (st != FA_OK) return st;
+  st = check_common(B, H, Nk, d, scale, FA_BF16);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_MISALIGNED;
+  if (static_cast<long long>(B) * H * Nq > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  const SplitPlan sp = split_plan(Nk, num_splits);
+  const SplitWs w = splitkv_ws(B, H, Nq, d, sp.n_split);
+  if (!workspace || workspace_bytes < w.total ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FA_ERR_WORKSPACE;
+  fa::Launch L;
+  st = device_context(stream, &L);
+  if (st != FA_OK) return st;
+  const int BH = B * H;
+  st = get_encoder();
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if ((st = make_map(&tq, q, BH, Nq, d)) != FA_OK) return st;
+  if ((st = make_map(&tk, k, BH, Nk, d)) != FA_OK) return st;
+  if ((st = make_map(&tv, v, BH, Nk, d)) != FA_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const fa::SplitKv sk{Nk, Nk - Nq, sp.n_split, sp.kt_per, reinterpret_cast<float*>(ws),
+                       reinterpret_cast<float*>(ws + w.lse_off)};
+  cudaError_t e = fa::launch_fwd_splitkv_sm100(tq, tk, tv, BH, Nq, d, scale, causal ? 1 : 0, sk, L);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = fa::launch_splitkv_combine(sk.part_o, sk.part_lse, o, lse, sp.n_split, BH * Nq, d, L);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
 fa_status fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
                       const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                       float scale, int causal, void* workspace, size_t workspace_bytes,

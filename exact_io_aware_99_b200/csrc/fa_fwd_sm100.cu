@@ -177,12 +177,38 @@ __device__ __forceinline__ void item_plan(int idx, int n_t, int BH, int group, i
   }
 }
 
-template <int D, bool CAUSAL, bool BS>
+__device__ __forceinline__ int floor_div(int a, int b) {
+  return a >= 0 ? a / b : -((-a + b - 1) / b);
+}
+
+// Split-KV items (decode): item idx = (tile pair item, split) with the split
+// fastest.  The split covers key tiles [t0, t0 + kt_per) of the N_k keys;
+// tile x visits the ones it sees (causal: keys <= query + coff, coff =
+// N_k - N_q, so the last query sees every key).
+template <bool CAUSAL>
+__device__ __forceinline__ void split_plan(int idx, int n_t, int BH, int group,
+                                           const SplitKv& sk, int& bh, int& pair, int& t0,
+                                           int (&n_x)[2]) {
+  decode_item<CAUSAL>(idx / sk.n_split, n_t, BH, group, bh, pair, n_x);
+  const int n_kt = (sk.Nk + kBN - 1) / kBN;
+  t0 = (idx % sk.n_split) * sk.kt_per;
+  const int t1 = min(t0 + sk.kt_per, n_kt);
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int qt = 2 * pair + x;
+    int end = t1;
+    if (CAUSAL) end = min(t1, floor_div(qt * kBM + kBM - 1 + sk.coff, kBN) + 1);
+    n_x[x] = qt >= n_t ? 0 : max(0, end - t0);
+  }
+}
+
+template <int D, bool CAUSAL, bool BS, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                float* __restrict__ lse, int N, int BH, int group, float scale_log2,
-               const uint8_t* __restrict__ bmask, int mask_heads, int H, WaitCtl ctl) {
+               const uint8_t* __restrict__ bmask, int mask_heads, int H, SplitKv sk,
+               WaitCtl ctl) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -211,7 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int n_t = (N + kBN - 1) / kBN;  // query tiles == key tiles
+  // Query tiles (== key tiles, except for split-KV launches where the N_k
+  // keys are counted by SplitKv).
+  const int n_t = (N + kBN - 1) / kBN;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -300,7 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         int bh, pair, n_x[2];
         ItemTiles<CAUSAL> tiles;
-        item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
+        int t0 = 0;  // first key tile of a split-KV item
+        if (SPLIT)
+          split_plan<CAUSAL>(idx, n_t, BH, group, sk, bh, pair, t0, n_x);
+        else
+          item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
         const int n_max = max(n_x[0], n_x[1]);
         if (n_max > 0) {
           // Q of this item replaces the previous item's once its S MMAs are done.
@@ -318,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++q_issued;
           TileCursor cur(n_t);
           for (int j = 0; j < n_max; ++j, ++kv) {
-            const int jt = BS ? cur.next(tiles) : j;  // key tile of the step
+            const int jt = BS ? cur.next(tiles) : t0 + j;  // key tile of the step
             const int s = static_cast<int>(kv % C::NST);
             const uint32_t u = kv / C::NST;
             if (kv >= C::NST && !wait(k_empty + s, (u - 1) & 1)) {
@@ -436,7 +468,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (idx < 0) break;
       int bh, pair, n_x[2];
       ItemTiles<CAUSAL> tiles;
-      item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
+      int t0 = 0;  // first key tile of a split-KV item
+        if (SPLIT)
+          split_plan<CAUSAL>(idx, n_t, BH, group, sk, bh, pair, t0, n_x);
+        else
+          item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
       const int n_max = max(n_x[0], n_x[1]);
       if (n_max == 0) continue;  // block mask hides the whole item
       const int r0 = static_cast<int>(kv_base);
@@ -498,18 +534,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (idx < 0) break;
       int bh, pair, n_x[2];
       ItemTiles<CAUSAL> tiles;
-      item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
+      int t0 = 0;  // first key tile of a split-KV item
+        if (SPLIT)
+          split_plan<CAUSAL>(idx, n_t, BH, group, sk, bh, pair, t0, n_x);
+        else
+          item_plan<CAUSAL, BS>(idx, n_t, BH, group, H, bmask, mask_heads, bh, pair, n_x, tiles);
       const int n_kv = n_x[x];
       const int qt_x = 2 * pair + x;
       const int q_idx = qt_x * kBM + r;
+      // Split-KV launches write this split's partial (O normalised over the
+      // split's keys, fp32, and its LSE) for the combine kernel.
+      const size_t prow =
+          SPLIT ? (static_cast<size_t>(idx % sk.n_split) * BH + bh) * N + q_idx : 0;
       if (n_kv == 0) {
-        // The block mask hides every key from this tile: O = 0, LSE = -inf.
-        // (Dense launches only get here for a tile past N: nothing to write.)
+        // No visible key for this tile (block mask, or a split past the
+        // causal limit): O = 0, LSE = -inf.  (Dense launches only get here
+        // for a tile past N: nothing to write.)
         if (q_idx < N) {
-          uint4* orow = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
+          if (SPLIT) {
+            float4* prw = reinterpret_cast<float4*>(sk.part_o + prow * D);
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
-          lse[static_cast<size_t>(bh) * N + q_idx] = -INFINITY;
+            for (int c = 0; c < D / 4; ++c) prw[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            sk.part_lse[prow] = -INFINITY;
+          } else {
+            uint4* orow =
+                reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+            lse[static_cast<size_t>(bh) * N + q_idx] = -INFINITY;
+          }
         }
         continue;
       }
@@ -517,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       TileCursor cur(n_t);
       for (int j = 0; j < n_kv; ++j) {
-        const int jt = BS ? cur.next(tiles) : j;  // key tile of the step
+        const int jt = BS ? cur.next(tiles) : t0 + j;  // key tile of the step
         if (!wait_all(s_full + x, (s_base + j) & 1, abort, ctl, kSiteFwdSoftmax)) {
           ok = false;
           break;
@@ -544,11 +597,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const int kv0 = jt * kBN;
-        const bool act = !BS || tiles.active(x, jt);  // false: the mask hides the whole step
-        const bool diag = CAUSAL && (BS ? jt == qt_x : j == n_kv - 1);
-        const bool masked = !act || diag || kv0 + kBN > N;
-        const int lim =
-            !act ? 0 : (masked ? min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN) : kBN);
+        bool masked;
+        int lim;
+        if (SPLIT) {
+          // N_k keys, query q sees keys <= q + coff when causal
+          masked = (CAUSAL && kv0 + kBN - 1 > qt_x * kBM + sk.coff) || kv0 + kBN > sk.Nk;
+          lim = masked ? min(sk.Nk - kv0, CAUSAL ? (q_idx + sk.coff - kv0 + 1) : kBN) : kBN;
+        } else {
+          const bool act = !BS || tiles.active(x, jt);  // false: the mask hides the whole step
+          const bool diag = CAUSAL && (BS ? jt == qt_x : j == n_kv - 1);
+          masked = !act || diag || kv0 + kBN > N;
+          lim = !act ? 0 : (masked ? min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN) : kBN);
+        }
         if (masked) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
@@ -625,25 +685,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         // l = 0 only for a row the block mask hides completely: O = 0.
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
         const bool valid = q_idx < N;
-        uint4* orow = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
+        const float lse_row = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (SPLIT) {
+          float4* prw = reinterpret_cast<float4*>(sk.part_o + prow * D);
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t o16[16];
-          tmem_ld16(lane_base + col_o + c * 16, o16);
-          tmem_wait_ld();
-          uint32_t pkd[8];
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o16[16];
+            tmem_ld16(lane_base + col_o + c * 16, o16);
+            tmem_wait_ld();
+            if (valid)
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            pkd[e] = pack_bf16(__uint_as_float(o16[2 * e]) * inv_l,
-                               __uint_as_float(o16[2 * e + 1]) * inv_l);
-          if (valid) {
-            orow[2 * c] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
-            orow[2 * c + 1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+              for (int e = 0; e < 4; ++e)
+                prw[4 * c + e] = make_float4(__uint_as_float(o16[4 * e]) * inv_l,
+                                             __uint_as_float(o16[4 * e + 1]) * inv_l,
+                                             __uint_as_float(o16[4 * e + 2]) * inv_l,
+                                             __uint_as_float(o16[4 * e + 3]) * inv_l);
           }
+          if (valid) sk.part_lse[prow] = lse_row;
+        } else {
+          uint4* orow =
+              reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o16[16];
+            tmem_ld16(lane_base + col_o + c * 16, o16);
+            tmem_wait_ld();
+            uint32_t pkd[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              pkd[e] = pack_bf16(__uint_as_float(o16[2 * e]) * inv_l,
+                                 __uint_as_float(o16[2 * e + 1]) * inv_l);
+            if (valid) {
+              orow[2 * c] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+              orow[2 * c + 1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+            }
+          }
+          if (valid) lse[static_cast<size_t>(bh) * N + q_idx] = lse_row;
         }
-        if (valid)
-          lse[static_cast<size_t>(bh) * N + q_idx] =
-              l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         // The next item's first P V (accumulate off) overwrites O_x only
         // after this warpgroup's next P, so the loads above are complete.
         tc_fence_before();
@@ -662,20 +740,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool BS>
+template <int D, bool CAUSAL, bool BS, bool SPLIT>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                    float* lse, int BH, int N, float scale, const BlockMaskArg& bm,
-                   const Launch& L) {
+                   const SplitKv& sk, const Launch& L) {
   using C = Cfg<D>;
   static bool configured = false;
   if (!configured) {
     // The register split above assumes the kernel was compiled to exactly
     // kLaunchRegs per thread; with fewer, the increase would wait forever.
     cudaFuncAttributes fattr;
-    cudaError_t e = cudaFuncGetAttributes(&fattr, fwd_kernel<D, CAUSAL, BS>);
+    cudaError_t e = cudaFuncGetAttributes(&fattr, fwd_kernel<D, CAUSAL, BS, SPLIT>);
     if (e != cudaSuccess) return e;
     if (fattr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(fwd_kernel<D, CAUSAL, BS>,
+    e = cudaFuncSetAttribute(fwd_kernel<D, CAUSAL, BS, SPLIT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
@@ -683,22 +761,23 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   const int n_t = (N + kBM - 1) / kBM;
   const int n_pair = (n_t + 1) / 2;
   // Heads per group: the operands every item of a head re-reads are K and V
-  // (4 N d bytes per head); a group's K and V stay within the L2 share
+  // (4 N_k d bytes per head); a group's K and V stay within the L2 share
   // (64 MB causal, 32 MB otherwise) while Q and O stream through.  Causal
   // launches need the large groups to keep the longest-first order global
   // enough that the last items are short ones (with 12-head groups the final
   // group's long items started last and left ~13% of the SMs idle at the end
   // of a causal N = 4096 launch).
-  const long long per_head = 4LL * N * D;
+  const long long per_head = 4LL * sk.Nk * D;
   int group = static_cast<int>(l2_group_bytes(CAUSAL) / (per_head > 0 ? per_head : 1));
   group = group < 1 ? 1 : (group > BH ? BH : group);
-  const long long blocks = static_cast<long long>(BH) * n_pair;
+  const long long blocks = static_cast<long long>(BH) * n_pair * (SPLIT ? sk.n_split : 1);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};
-  fwd_kernel<D, CAUSAL, BS><<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
-      tq, tk, tv, static_cast<__nv_bfloat16*>(o), lse, N, BH, group, scale_log2, bm.mask,
-      bm.mask_heads, bm.H, ctl);
+  fwd_kernel<D, CAUSAL, BS, SPLIT>
+      <<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
+          tq, tk, tv, static_cast<__nv_bfloat16*>(o), lse, N, BH, group, scale_log2, bm.mask,
+          bm.mask_heads, bm.H, sk, ctl);
   return cudaGetLastError();
 }
 
@@ -707,11 +786,25 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      void* o, float* lse, int BH, int N, float scale, int causal,
                      const BlockMaskArg* bm, const Launch& L) {
   const BlockMaskArg none{nullptr, 1, 1};
+  const SplitKv dense{N, 0, 1, (N + kBN - 1) / kBN, nullptr, nullptr};
   if (bm && bm->mask)
-    return causal ? launch<D, true, true>(tq, tk, tv, o, lse, BH, N, scale, *bm, L)
-                  : launch<D, false, true>(tq, tk, tv, o, lse, BH, N, scale, *bm, L);
-  return causal ? launch<D, true, false>(tq, tk, tv, o, lse, BH, N, scale, none, L)
-                : launch<D, false, false>(tq, tk, tv, o, lse, BH, N, scale, none, L);
+    return causal ? launch<D, true, true, false>(tq, tk, tv, o, lse, BH, N, scale, *bm, dense, L)
+                  : launch<D, false, true, false>(tq, tk, tv, o, lse, BH, N, scale, *bm, dense,
+                                                  L);
+  return causal ? launch<D, true, false, false>(tq, tk, tv, o, lse, BH, N, scale, none, dense, L)
+                : launch<D, false, false, false>(tq, tk, tv, o, lse, BH, N, scale, none, dense,
+                                                 L);
+}
+
+template <int D>
+cudaError_t launch_split_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           int BH, int Nq, float scale, int causal, const SplitKv& sk,
+                           const Launch& L) {
+  const BlockMaskArg none{nullptr, 1, 1};
+  return causal ? launch<D, true, false, true>(tq, tk, tv, nullptr, nullptr, BH, Nq, scale, none,
+                                               sk, L)
+                : launch<D, false, false, true>(tq, tk, tv, nullptr, nullptr, BH, Nq, scale, none,
+                                                sk, L);
 }
 
 }  // namespace fwd
@@ -726,6 +819,21 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
       return fwd::launch_d<80>(tq, tk, tv, o, lse, BH, N, scale, causal, bm, L);
     case 128:
       return fwd::launch_d<128>(tq, tk, tv, o, lse, BH, N, scale, causal, bm, L);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_fwd_splitkv_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                     const CUtensorMap& tv, int BH, int Nq, int d, float scale,
+                                     int causal, const SplitKv& sk, const Launch& L) {
+  switch (d) {
+    case 64:
+      return fwd::launch_split_d<64>(tq, tk, tv, BH, Nq, scale, causal, sk, L);
+    case 80:
+      return fwd::launch_split_d<80>(tq, tk, tv, BH, Nq, scale, causal, sk, L);
+    case 128:
+      return fwd::launch_split_d<128>(tq, tk, tv, BH, Nq, scale, causal, sk, L);
     default:
       return cudaErrorInvalidValue;
   }

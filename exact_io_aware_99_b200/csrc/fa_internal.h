@@ -61,12 +61,35 @@ struct BlockMaskArg {
   int H;                // heads per batch entry
 };
 
+// Split-KV forward (decode): N_q queries against N_k keys, the key tiles of
+// every (head, query tile pair) split into n_split ranges of kt_per tiles;
+// each range writes a partial O (fp32, normalised over its keys) and LSE to
+// part_o [n_split, BH, N_q, d] / part_lse [n_split, BH, N_q], merged by
+// launch_splitkv_combine.  coff = N_k - N_q (causal: query i sees keys
+// j <= i + coff).  Dense launches use {N, 0, 1, ceil(N / 128), null, null}.
+struct SplitKv {
+  int Nk, coff, n_split, kt_per;
+  float* part_o;
+  float* part_lse;
+};
+
 // --- bf16 tensor-core path (fa_fwd_sm100.cu, fa_bwd_sm100.cu) -------------
 // Tensor maps describe a [BH, N, d] bf16 tensor as 3-D {d, N, BH} with a
 // {64, 128, 1} box and 128-byte swizzle.
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              void* o, float* lse, int BH, int N, int d, float scale, int causal,
                              const BlockMaskArg* bm, const Launch& L);
+
+// Split-KV forward: tq has N_q rows per head, tk / tv N_k (sk.Nk) rows.
+cudaError_t launch_fwd_splitkv_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                     const CUtensorMap& tv, int BH, int Nq, int d, float scale,
+                                     int causal, const SplitKv& sk, const Launch& L);
+
+// Merge of the split-KV partials: LSE = m + ln sum_s e^(LSE_s - m),
+// O = sum_s e^(LSE_s - LSE) O_s (bf16 out); rows with every LSE_s = -inf give
+// O = 0, LSE = -inf.  rows = BH * N_q.
+cudaError_t launch_splitkv_combine(const float* part_o, const float* part_lse, void* o,
+                                   float* lse, int n_split, int rows, int d, const Launch& L);
 
 // Backward: the dK/dV kernel then the dQ kernel, both in stream order.
 // dvec and lse2 are the preprocess outputs ([BH, Np] fp32, Np = N rounded up

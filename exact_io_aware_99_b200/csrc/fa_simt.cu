@@ -277,6 +277,46 @@ __global__ void selftest_wait_kernel(WaitCtl ctl) {
   __syncthreads();
 }
 
+// Merge of split-KV partials, one warp per output row: LSE = m + ln S,
+// S = sum_s e^(LSE_s - m), m = max_s LSE_s, and O = sum_s e^(LSE_s - m) O_s / S
+// ("FlashAttention-2" review: the online-softmax merge of running max and
+// sum, applied across the key splits).  Rows whose splits all saw no key
+// (every LSE_s = -inf) get O = 0 and LSE = -inf.
+__global__ void splitkv_combine_kernel(const float* __restrict__ part_o,
+                                       const float* __restrict__ part_lse,
+                                       __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                                       int n_split, int rows, int d) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= rows) return;
+  float m = -INFINITY;
+  for (int s = 0; s < n_split; ++s)
+    m = fmaxf(m, part_lse[static_cast<size_t>(s) * rows + row]);
+  __nv_bfloat16* orow = o + static_cast<size_t>(row) * d;
+  if (m == -INFINITY) {
+    for (int c = lane; c < d; c += 32) orow[c] = __float2bfloat16(0.f);
+    if (lane == 0) lse[row] = -INFINITY;
+    return;
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // columns lane, lane + 32, lane + 64, lane + 96
+  float tot = 0.f;
+  for (int s = 0; s < n_split; ++s) {
+    const float ls = part_lse[static_cast<size_t>(s) * rows + row];
+    if (ls == -INFINITY) continue;
+    const float w = expf(ls - m);
+    tot += w;
+    const float* prow = part_o + (static_cast<size_t>(s) * rows + row) * d;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (lane + 32 * e < d) acc[e] += w * prow[lane + 32 * e];
+  }
+  const float inv = 1.f / tot;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (lane + 32 * e < d) orow[lane + 32 * e] = __float2bfloat16(acc[e] * inv);
+  if (lane == 0) lse[row] = m + logf(tot);
+}
+
 }  // namespace simt
 
 static int blocks_for(size_t work, int per_block) {
@@ -334,6 +374,16 @@ cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* ls
     simt::bwd_preprocess_kernel<float><<<blocks, threads, 0, L.stream>>>(
         static_cast<const float*>(o), static_cast<const float*>(dO), lse, dvec, lse2, BH, N, Np,
         d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_splitkv_combine(const float* part_o, const float* part_lse, void* o,
+                                   float* lse, int n_split, int rows, int d, const Launch& L) {
+  if (d > 128) return cudaErrorInvalidValue;
+  const int threads = 256;
+  const int blocks = blocks_for(static_cast<size_t>(rows) * 32, threads);
+  simt::splitkv_combine_kernel<<<blocks, threads, 0, L.stream>>>(
+      part_o, part_lse, static_cast<__nv_bfloat16*>(o), lse, n_split, rows, d);
   return cudaGetLastError();
 }
 

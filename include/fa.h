@@ -188,6 +188,44 @@ FA_API fa_status fa_backward_blocksparse(const void* q, const void* k, const voi
                                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_forward_splitkv -- bf16 forward for decoding: N_q new queries against a
+ * cache of N_k >= 1 keys/values, the key range split across CTAs.  Each
+ * (head, query tile pair, key split) computes a partial O and LSE over its
+ * keys with the online softmax; a second kernel merges the partials by the
+ * same running-max / running-sum rule ("FlashAttention-2: Faster Attention
+ * with Better Parallelism and Work Partitioning" review: core-algorithm
+ * answer, (2) forward pass step 2, and its answer on FlashAttention's Split-K
+ * scheme, where K and V are split across workers whose partial results are
+ * combined).  Splitting the keys gives a few-query problem enough parallel
+ * work to keep every SM reading K and V.
+ *   q, o        [B, H, N_q, d] bf16;  lse [B, H, N_q] fp32 (natural log).
+ *   k, v        [B, H, N_k, d] bf16.
+ *   causal      0: every query sees every key; 1: the queries are the last
+ *               N_q positions: query i sees keys j <= i + (N_k - N_q).  Rows
+ *               that see no key (only when N_q > N_k) get O = 0, LSE = -inf.
+ *   num_splits  >= 1 key ranges per (head, query tile pair); clamped to the
+ *               number of 128-key tiles.  fa_splitkv_default_splits picks one.
+ *   workspace   device scratch of fa_splitkv_workspace_size(...) bytes,
+ *               256-byte aligned (fp32 partials), owned by the caller;
+ *               concurrent calls must not share it.
+ * d in {64, 80, 128}.  Errors as fa_forward; FA_ERR_WORKSPACE for a missing,
+ * small or misaligned workspace.  Two kernels in stream order.
+ */
+FA_API fa_status fa_forward_splitkv(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int B, int H, int Nq, int Nk, int d,
+                                    float scale, int causal, int num_splits, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* Key splits for fa_forward_splitkv that give about two work items per SM of
+ * the current device (1 .. ceil(N_k / 128)); 0 for invalid sizes. */
+FA_API int fa_splitkv_default_splits(int B, int H, int Nq, int Nk);
+
+/* Workspace bytes fa_forward_splitkv needs for these sizes and num_splits:
+ * fp32 partial O and LSE for every split, each rounded up to 256 bytes;
+ * 0 for invalid arguments. */
+FA_API size_t fa_splitkv_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits);
+
+/*
  * fa_backward_noalloc -- the bf16 backward of fa_backward, for callers that
  * cannot allocate device memory or hand over a workspace: code whose device
  * memory is entirely owned by another allocator, plugins and callbacks that
