@@ -344,11 +344,150 @@ def run_ours(args, peaks, peak_kind):
 
 # ------------------------------------------------------------- CPU oracle
 
+def run_decode(args, peaks, peak_kind):
+    """Split-KV decode workload: forward only, N_q queries against N_k keys.
+    Bound by HBM (K and V are read once per query tile pair), so the roofline
+    is GB/s of algorithmic bytes against the measured copy bandwidth."""
+    import exact_io_aware_99_b200 as fa
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = workloads.WORKLOADS[args.workload]
+    B, H, Nq, Nk, d = w.B, w.H, w.N, w.nk, w.d
+    x = workloads.make_decode_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), device=dev, dtype=torch.float32)
+    splits = args.splits if args.splits else fa.fa_splitkv_default_splits(B, H, Nq, Nk)
+    wbytes = fa.fa_splitkv_workspace_size(B, H, Nq, Nk, d, splits)
+    wsbuf = torch.empty(wbytes, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def fwd():
+        fa.fa_forward_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, w.scale, w.causal, splits, wsbuf,
+                              wbytes, sp)
+
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        fwd()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    st, site = fa.fa_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError(f"device wait timed out (site {site:#x})")
+    ms = a.elapsed_time(b) / args.steps
+    if ws > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    flops = perf.decode_flops(B, H, Nq, Nk, d, w.causal)
+    nbytes = perf.decode_bytes(B, H, Nq, Nk, d)
+    value = ws * flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+        ho = torch.empty_like(hq).pin_memory()
+        hlse = torch.empty((B, H, Nq), dtype=torch.float32).pin_memory()
+        bi = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        bo = sum(t.numel() * t.element_size() for t in (ho, hlse))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            fwd()
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ne = max(3, min(args.steps, 10))
+        ea.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        eb.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = ea.elapsed_time(eb) / ne
+        e2e = {"value": round(ws * flops / (e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e_ms, 4)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        from oracle.decode import rect_forward
+        cores = os.cpu_count() or 1
+        x1 = workloads.make_decode_inputs(w, B=1)
+        n, t0 = 0, time.perf_counter()
+        while True:
+            h = n % H
+            rect_forward(x1["q"][0, h], x1["k"][0, h], x1["v"][0, h], w.scale, w.causal)
+            n += 1
+            if time.perf_counter() - t0 >= args.cpu_seconds:
+                break
+        el = time.perf_counter() - t0
+        cpu = {"value": round(n * perf.decode_flops(1, 1, Nq, Nk, d, w.causal) / el / 1e12, 6),
+               "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n} head(s) of {w.name}, forward, fp64 numpy on the host ({el:.1f} s)"}
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    hbm = float(peaks.get("hbm_gbs", 6534.8))
+    peak = float(peaks["bf16_tflops"])
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded iid N(0,1), rounded to bf16)",
+        "config": {"workload": w.describe(), "B": B, "H": H, "N_q": Nq, "N_k": Nk, "d": d,
+                   "causal": w.causal, "passes": "fwd (split-KV decode)", "num_splits": splits,
+                   "l2": "K/V ~%.2f GB > 126 MB L2 (no flush needed)"
+                         % (2 * B * H * Nk * d * 2 / 1e9),
+                   "parallelism": f"{ws} independent replicas" if ws > 1 else "single GPU"},
+        "fwd_tflops": round(value / ws, 3), "fwd_frac_of_peak": round(value / ws / peak, 4),
+        "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs {hbm}, bf16_tflops {peak})",
+        "roofline": {"kernel": "fa_forward_splitkv (split forward + combine)", "bound": "hbm",
+                     "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(gbs / hbm, 4), "traffic": None,
+                     "algorithmic_bytes": nbytes},
+        "gpu_launches": 2 * args.steps,
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                   "reasons": clk["reasons"], "samples": clk["samples"]},
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+
+
 def step_flop_counts(w, B=None, H=None):
     """Algorithmic forward and backward FLOPs of one step of workload w
     (visible pairs only for a block-sparse workload)."""
     B = w.B if B is None else B
     H = w.H if H is None else H
+    if w.nk:
+        return perf.decode_flops(B, H, w.N, w.nk, w.d, w.causal), 0.0
     m = workloads.block_mask(w)
     if m is not None:
         return (perf.fwd_flops_masked(B, H, w.N, w.d, w.causal, m),
@@ -360,6 +499,10 @@ def oracle_head_step(w, x, h):
     """Forward and backward of head h of x on the fp64 oracle (the
     block-sparse oracle for a block-sparse workload)."""
     import oracle
+    if w.nk:
+        from oracle.decode import rect_forward
+        rect_forward(x["q"][0, h], x["k"][0, h], x["v"][0, h], w.scale, w.causal)
+        return
     qh, kh, vh, doh = (x[n][0, h] for n in ("q", "k", "v", "do"))
     m = workloads.block_mask(w)
     if m is not None:
@@ -395,7 +538,8 @@ def run_reference(args):
     if rank != 0:
         return None
     w = workloads.WORKLOADS[args.workload]
-    x = workloads.make_inputs(w, with_grad_out=True, B=1)
+    x = (workloads.make_decode_inputs(w, B=1) if w.nk
+         else workloads.make_inputs(w, with_grad_out=True, B=1))
     per_head = sum(step_flop_counts(w, B=1, H=1))
 
     def step(i):
@@ -415,7 +559,7 @@ def run_reference(args):
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.describe(), "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                       "causal": w.causal, "passes": "fwd+bwd"},
+                       "causal": w.causal, "passes": "fwd" if w.nk else "fwd+bwd"},
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
                              "kind": "oracle", "sample": sample},
@@ -482,6 +626,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true", help="print the TFLOP/s-vs-N sweep instead")
+    ap.add_argument("--splits", type=int, default=0,
+                    help="key splits for a decode workload (0: the library's default)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -491,6 +637,8 @@ def main(argv=None):
     elif args.sweep:
         run_sweep(args, peaks)
         return
+    elif workloads.WORKLOADS[args.workload].nk:
+        line = run_decode(args, peaks, kind)
     else:
         line = run_ours(args, peaks, kind)
     if line is not None:

@@ -369,7 +369,10 @@ int fa_splitkv_default_splits(int B, int H, int Nq, int Nk) {
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = static_cast<long long>(B) * H * (((Nq + 127) / 128 + 1) / 2);
-  const long long want = (2LL * sms + items - 1) / items;  // about two items per SM
+  // About four items per SM: the launch is bound by reading K and V, and
+  // more, shorter items shrink the idle tail of the last wave; the partials
+  // the combine kernel reads grow with the split count (4 N_q d bytes each).
+  const long long want = (4LL * sms + items - 1) / items;
   const int n_kt = (Nk + 127) / 128;
   const int s = static_cast<int>(want < 1 ? 1 : (want > n_kt ? n_kt : want));
   return split_plan(Nk, s).n_split;

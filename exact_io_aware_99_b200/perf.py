@@ -68,3 +68,23 @@ def fwd_flops_masked(B: int, H: int, N: int, d: int, causal: bool, block_mask) -
 
 def bwd_flops_masked(B: int, H: int, N: int, d: int, causal: bool, block_mask) -> float:
     return 2.5 * fwd_flops_masked(B, H, N, d, causal, block_mask)
+
+
+def decode_pairs(Nq: int, Nk: int, causal: bool) -> float:
+    """Visible (query, key) pairs of N_q queries that are the last N_q of N_k
+    positions (causal: query i sees keys j <= i + N_k - N_q)."""
+    if not causal:
+        return float(Nq) * Nk
+    total = 0.0
+    for i in range(Nq):
+        total += max(0, min(Nk, i + Nk - Nq + 1))
+    return total
+
+
+def decode_flops(B: int, H: int, Nq: int, Nk: int, d: int, causal: bool) -> float:
+    return 4.0 * d * B * H * decode_pairs(Nq, Nk, causal)
+
+
+def decode_bytes(B: int, H: int, Nq: int, Nk: int, d: int, elem: int = 2) -> float:
+    """Q read + O written (N_q rows), K and V read (N_k rows), LSE written."""
+    return 2.0 * B * H * Nq * d * elem + 2.0 * B * H * Nk * d * elem + 4.0 * B * H * Nq

@@ -16,6 +16,9 @@ Workloads (shapes are [B, H, N, d], d fastest):
   own plus key tiles 0 and 1 (a local window with global tokens, the hybrid
   local + global pattern the FlashAttention-2 review names for sparse
   attention); 128 x 128 tiles, one mask for all heads, ~8.6 % of the pairs.
+* ``decode_d128`` B8 H16, 128 new queries against a 16384-entry key/value
+  cache, d128, bf16, causal (the queries are the last 128 positions),
+  forward only, split-KV.
 * ``gpt3_d80``    B8 H32 N2048 d80, bf16, causal, forward+backward; Q, K, V
   are projections X.W of a unit-normal activation X [B, N, 2560] through
   three independent N(0, 0.02^2) [2560, 2560] weights, then split into
@@ -49,6 +52,7 @@ class Workload:
     projected: bool = False   # Q/K/V = X.W (GPT-3 shaped layer)
     hidden: int = 0
     mask: str = ""            # block-sparse pattern name ("" = dense)
+    nk: int = 0               # keys when they differ from the N queries (decode)
 
     @property
     def scale(self) -> float:
@@ -66,7 +70,8 @@ class Workload:
         pas = "fwd+bwd" if self.backward else "fwd"
         cz = "causal" if self.causal else "non-causal"
         bs = f" block-sparse {self.mask}" if self.mask else ""
-        return (f"{self.name}: B{self.B} H{self.H} N{self.N} d{self.d} "
+        n = f"N_q{self.N} N_k{self.nk}" if self.nk else f"N{self.N}"
+        return (f"{self.name}: B{self.B} H{self.H} {n} d{self.d} "
                 f"{self.dtype} {cz}{bs} {pas}")
 
 
@@ -80,6 +85,7 @@ WORKLOADS: Dict[str, Workload] = {
                  projected=True, hidden=2560),
         Workload("bsparse_d128", 5, 1, 16, 16384, 128, "bf16", False, True,
                  mask="local4_global2"),
+        Workload("decode_d128", 6, 8, 16, 128, 128, "bf16", True, False, nk=16384),
     ]
 }
 
@@ -160,4 +166,16 @@ def random_case(B: int, H: int, N: int, d: int, seed: int,
     for name in names:
         x = torch.randn(B, H, N, d, generator=g, dtype=torch.float32) * std
         out[name] = round_to(x, dtype)
+    return out
+
+
+def make_decode_inputs(w: Workload, B: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Seeded CPU inputs of a decode workload: q [B, H, N, d] and k, v
+    [B, H, nk, d], iid N(0, 1) rounded to the storage dtype."""
+    B = w.B if B is None else B
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    dt = w.torch_dtype
+    out = {"q": round_to(torch.randn(B, w.H, w.N, w.d, generator=g), dt)}
+    for name in ("k", "v"):
+        out[name] = round_to(torch.randn(B, w.H, w.nk, w.d, generator=g), dt)
     return out
