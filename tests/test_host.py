@@ -160,3 +160,55 @@ def test_masked_flop_counts_reduce_to_the_dense_ones():
     mh = np.zeros((2, 3, 3), bool)
     mh[0, 1, 0] = mh[1, 2, 2] = True           # tile 2 is 44 rows: 44 x 44
     assert perf.fwd_flops_masked(1, 2, 300, 8, False, mh) == 4 * 8 * (128 * 128 + 44 * 44)
+
+
+def test_splitkv_workspace_formula_and_split_clamping():
+    fa = _lib()
+    up = lambda x: (x + 255) // 256 * 256
+    # 3 splits of a 1000-key cache (8 key tiles -> ranges of 3, 3, 2 tiles)
+    B, H, Nq, Nk, d = 2, 3, 5, 1000, 80
+    rows = 3 * B * H * Nq
+    assert fa.fa_splitkv_workspace_size(B, H, Nq, Nk, d, 3) == up(rows * d * 4) + up(rows * 4)
+    # more splits than key tiles clamp to one tile per split; 5 requested
+    # splits of 8 tiles become ranges of 2 tiles, i.e. 4 splits
+    assert fa.fa_splitkv_workspace_size(1, 1, 16, 256, 128, 10) == \
+        fa.fa_splitkv_workspace_size(1, 1, 16, 256, 128, 2)
+    assert fa.fa_splitkv_workspace_size(1, 1, 16, 1024, 128, 5) == \
+        fa.fa_splitkv_workspace_size(1, 1, 16, 1024, 128, 4)
+    for bad in ((0, 1, 1, 1, 64, 1), (1, 1, 0, 1, 64, 1), (1, 1, 1, 0, 64, 1),
+                (1, 1, 1, 1, 64, 0), (1, 1, 1, 1, 200, 1)):
+        assert fa.fa_splitkv_workspace_size(*bad) == 0
+    assert 1 <= fa.fa_splitkv_default_splits(1, 1, 1, 16384) <= 128
+    assert fa.fa_splitkv_default_splits(1, 1, 1, 100) == 1
+
+
+def test_new_entry_points_reject_bad_arguments_before_any_device_call():
+    fa = _lib()
+    # split-KV: null pointer, zero splits, bad head dim
+    st = fa.fa_forward_splitkv(0, A, A, A, A, 1, 1, 4, 256, 64, 0.1, 0, 1, A, 1 << 20,
+                               stream=0, check=False)
+    assert st == -1
+    st = fa.fa_forward_splitkv(A, A, A, A, A, 1, 1, 4, 256, 64, 0.1, 0, 0, A, 1 << 20,
+                               stream=0, check=False)
+    assert st == -1
+    st = fa.fa_forward_splitkv(A, A, A, A, A, 1, 1, 4, 256, 96, 0.1, 0, 1, A, 1 << 20,
+                               stream=0, check=False)
+    assert st == -2
+    # block-sparse: null mask, mask_heads neither 1 nor H
+    st = fa.fa_forward_blocksparse(A, A, A, A, A, 1, 2, 256, 64, 0.1, 0, None, 1, stream=0, check=False)
+    assert st == -1
+    st = fa.fa_forward_blocksparse(A, A, A, A, A, 1, 2, 256, 64, 0.1, 0, A, 3, stream=0, check=False)
+    assert st == -1
+    st = fa.fa_backward_blocksparse(A, A, A, A, A, A, A, A, A, 1, 2, 256, 64, 0.1, 0, A, 5,
+                                    A, 1 << 20, stream=0, check=False)
+    assert st == -1
+
+
+def test_decode_flop_and_byte_counts():
+    assert perf.decode_pairs(3, 7, True) == 5 + 6 + 7
+    assert perf.decode_pairs(5, 3, True) == 0 + 0 + 1 + 2 + 3
+    assert perf.decode_pairs(4, 9, False) == 36
+    # square causal decode = the dense causal pair count N (N + 1) / 2
+    assert perf.decode_pairs(300, 300, True) == 300 * 301 / 2
+    assert perf.decode_flops(2, 3, 4, 9, 16, False) == 4 * 16 * 2 * 3 * 36
+    assert perf.decode_bytes(1, 1, 2, 10, 8) == 2 * 2 * 8 * 2 + 2 * 10 * 8 * 2 + 4 * 2
