@@ -24,16 +24,21 @@ Workloads (shapes are [B, H, N, d], d fastest):
   three independent N(0, 0.02^2) [2560, 2560] weights, then split into
   32 heads of 80 (the GPT-3 2.7B layer shape named on the FlashAttention-2
   review page, section on results, GPT-3 2.7B end-to-end training).
+* ``fp8_causal_d128`` B4 H16 N4096 d128, E4M3 Q/K/V with one fp32
+  dequantisation factor per tensor, causal, forward only (the FP8 forward the
+  FlashAttention-2 review lists under future work, item (5)); the same shape
+  as ``causal_d128``.
 
 Every tensor is generated in fp32 on the CPU from ``torch.Generator`` seeded
 with ``1000 + index`` and then rounded (round-to-nearest-even) to the storage
-dtype, so the GPU and the oracle see the same bits.
+dtype, so the GPU and the oracle see the same bits.  E4M3 tensors are drawn
+the same way in fp32 and then quantised per tensor by ``quantize_e4m3``.
 """
 from __future__ import annotations
 
 import math
 from dataclasses import dataclass, field
-from typing import Dict, Optional
+from typing import Dict, Optional, Tuple
 
 import torch
 
@@ -46,7 +51,7 @@ class Workload:
     H: int
     N: int
     d: int
-    dtype: str          # "fp32" or "bf16"
+    dtype: str          # "fp32", "bf16" or "e4m3"
     causal: bool
     backward: bool
     projected: bool = False   # Q/K/V = X.W (GPT-3 shaped layer)
@@ -64,7 +69,8 @@ class Workload:
 
     @property
     def torch_dtype(self) -> torch.dtype:
-        return torch.float32 if self.dtype == "fp32" else torch.bfloat16
+        return {"fp32": torch.float32, "bf16": torch.bfloat16,
+                "e4m3": torch.float8_e4m3fn}[self.dtype]
 
     def describe(self) -> str:
         pas = "fwd+bwd" if self.backward else "fwd"
@@ -86,6 +92,7 @@ WORKLOADS: Dict[str, Workload] = {
         Workload("bsparse_d128", 5, 1, 16, 16384, 128, "bf16", False, True,
                  mask="local4_global2"),
         Workload("decode_d128", 6, 8, 16, 128, 128, "bf16", True, False, nk=16384),
+        Workload("fp8_causal_d128", 7, 4, 16, 4096, 128, "e4m3", True, False),
     ]
 }
 
@@ -179,3 +186,84 @@ def make_decode_inputs(w: Workload, B: Optional[int] = None) -> Dict[str, torch.
     for name in ("k", "v"):
         out[name] = round_to(torch.randn(B, w.H, w.nk, w.d, generator=g), dt)
     return out
+
+
+# Largest finite E4M3 value (1.75 * 2^8); the per-tensor quantisation maps
+# the tensor's largest magnitude onto it.
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: torch.Tensor) -> Tuple[torch.Tensor, float]:
+    """Per-tensor E4M3 quantisation of a float tensor (computed in fp32):
+    amax = max |x|, descale = amax / 448 and codes = RN(x * (448 / amax)),
+    each step one fp32 operation, the last through torch's float8_e4m3fn
+    conversion (round to nearest even); amax = 0 gives descale 1.  Returns
+    the codes as a contiguous uint8 tensor and the fp32 descale factor."""
+    xf = x.float()
+    amax = xf.abs().max() if xf.numel() else torch.tensor(0.0)
+    lim = torch.tensor(E4M3_MAX, dtype=torch.float32)
+    if float(amax) > 0.0:
+        inv = lim / amax
+        descale = float(amax / lim)
+    else:
+        inv = torch.tensor(1.0, dtype=torch.float32)
+        descale = 1.0
+    codes = (xf * inv).to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    return codes, descale
+
+
+def make_fp8_inputs(w: Workload, B: Optional[int] = None, H: Optional[int] = None,
+                    N: Optional[int] = None, seed: Optional[int] = None) -> Dict[str, object]:
+    """Seeded inputs of an E4M3 workload: q, k, v drawn iid N(0, 1) in fp32
+    [B, H, N, d] and quantised per tensor.  Returns {"q8", "k8", "v8"} (uint8
+    codes) and {"q_descale", "k_descale", "v_descale"} (floats)."""
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    N = w.N if N is None else N
+    g = torch.Generator(device="cpu").manual_seed(w.seed if seed is None else seed)
+    out: Dict[str, object] = {}
+    for name in ("q", "k", "v"):
+        codes, ds = quantize_e4m3(torch.randn(B, H, N, w.d, generator=g, dtype=torch.float32))
+        out[name + "8"] = codes
+        out[name + "_descale"] = ds
+    return out
+
+
+def fp8_random_case(B: int, H: int, N: int, d: int, seed: int,
+                    std: float = 1.0) -> Dict[str, object]:
+    """Small seeded E4M3 case (iid N(0, std^2), quantised per tensor)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    out: Dict[str, object] = {}
+    for name in ("q", "k", "v"):
+        codes, ds = quantize_e4m3(torch.randn(B, H, N, d, generator=g) * std)
+        out[name + "8"] = codes
+        out[name + "_descale"] = ds
+    return out
+
+
+def fp8_exact_case(B: int, H: int, N: int, d: int, seed: int) -> Dict[str, object]:
+    """E4M3 case whose probabilities are exact E4M3 values.
+
+    Every query row holds one or two entries of +-1 (code value; descale
+    1/2), every key entry is an integer in [-2, 2] (descale 2), so with the
+    attention scale ln 2 each score, in base-2 units, is an integer in
+    [-4, 4]: any probability taken against a reference maximum inside the
+    row's range is a power of two between 2^-8 and 2^8, which E4M3 holds
+    exactly.  V is iid N(0, 1) quantised per tensor.  Use scale = ln 2."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    q = torch.zeros(B, H, N, d)
+    nnz = torch.randint(1, 3, (B, H, N), generator=g)
+    pos = torch.randint(0, d, (B, H, N, 2), generator=g)
+    sgn = torch.randint(0, 2, (B, H, N, 2), generator=g).float() * 2 - 1
+    for t in range(2):
+        keep = (nnz > t).float()
+        q.scatter_add_(3, pos[..., t:t + 1], (sgn[..., t] * keep).unsqueeze(-1))
+    q = q.clamp(-1.0, 1.0)   # two hits on one position stay within +-1
+    k = torch.randint(-2, 3, (B, H, N, d), generator=g).float()
+    v8, v_ds = quantize_e4m3(torch.randn(B, H, N, d, generator=g))
+    return {
+        "q8": q.to(torch.float8_e4m3fn).view(torch.uint8).contiguous(),
+        "k8": k.to(torch.float8_e4m3fn).view(torch.uint8).contiguous(),
+        "v8": v8,
+        "q_descale": 0.5, "k_descale": 2.0, "v_descale": v_ds,
+    }
