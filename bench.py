@@ -131,6 +131,9 @@ KERNEL_SOURCES = {
             "exact_io_aware_99_b200/csrc/sm100.cuh", "exact_io_aware_99_b200/csrc/fa_internal.h"],
     "fwd": ["exact_io_aware_99_b200/csrc/fa_fwd_sm100.cu", "exact_io_aware_99_b200/csrc/sm100.cuh",
             "exact_io_aware_99_b200/csrc/fa_internal.h"],
+    "fwd8": ["exact_io_aware_99_b200/csrc/fa_fwd_fp8_sm100.cu",
+             "exact_io_aware_99_b200/csrc/fa_fp8.h", "exact_io_aware_99_b200/csrc/sm100.cuh",
+             "exact_io_aware_99_b200/csrc/fa_internal.h"],
 }
 
 
@@ -481,6 +484,136 @@ def run_decode(args, peaks, peak_kind):
     }
 
 
+def run_fp8(args, peaks, peak_kind):
+    """FP8 (E4M3) forward workload.  Its three E4M3 inputs (1 byte per
+    element) fit in L2, so L2 is flushed (a 256 MB write) before every timed
+    step and each step is timed by its own pair of events; the roofline is
+    the tensor pipe at the FP8 rate, twice the measured bf16 GEMM peak (the
+    nominal 4.5 / 2.25 PFLOP/s ratio)."""
+    import exact_io_aware_99_b200 as fa
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = workloads.WORKLOADS[args.workload]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    x = workloads.make_fp8_inputs(w)
+    q8, k8, v8 = (x[n].to(dev) for n in ("q8", "k8", "v8"))
+    ds = {n: torch.tensor([x[n + "_descale"]], device=dev, dtype=torch.float32)
+          for n in ("q", "k", "v")}
+    o = torch.empty((B, H, N, d), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def fwd():
+        fa.fa_forward_fp8(q8, k8, v8, ds["q"], ds["k"], ds["v"], o, lse, B, H, N, d, w.scale,
+                          w.causal, sp)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        fwd()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    st, site = fa.fa_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError(f"device wait timed out (site {site:#x})")
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    if ws > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    flops = perf.fwd_flops(B, H, N, d, w.causal)
+    value = ws * flops / (ms * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x[n].pin_memory() for n in ("q8", "k8", "v8"))
+        ho = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+        hlse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+        bi = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        bo = sum(t.numel() * t.element_size() for t in (ho, hlse))
+
+        def e2e_step():
+            q8.copy_(hq, non_blocking=True)
+            k8.copy_(hk, non_blocking=True)
+            v8.copy_(hv, non_blocking=True)
+            fwd()
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ne = max(3, min(args.steps, 10))
+        ea.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        eb.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = ea.elapsed_time(eb) / ne
+        e2e = {"value": round(ws * flops / (e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e_ms, 4)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    bf16_peak = float(peaks["bf16_tflops"])
+    peak = 2.0 * bf16_peak
+    achieved = value / ws
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic (seeded iid N(0,1) fp32, quantised per tensor to E4M3)",
+        "config": {"workload": w.describe(), "B": B, "H": H, "N": N, "d": d,
+                   "causal": w.causal, "passes": "fwd (FP8)",
+                   "l2": "flushed before every timed step (256 MB write; inputs %.0f MB < L2)"
+                         % (3 * B * H * N * d / 1e6),
+                   "parallelism": f"{ws} independent replicas" if ws > 1 else "single GPU"},
+        "fwd_tflops": round(achieved, 3),
+        "fwd_frac_of_bf16_peak": round(achieved / bf16_peak, 4),
+        "peak_source": (f"{peak_kind}: bf16_tflops {bf16_peak} x 2 (nominal FP8 / bf16 dense "
+                        f"ratio 4.5 / 2.25 PFLOP/s)"),
+        "roofline": {"kernel": "fwd_fp8_kernel", "bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": recorded_traffic("fwd8", args.workload),
+                     "algorithmic_flops": flops},
+        "gpu_launches": args.steps,
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                   "reasons": clk["reasons"], "samples": clk["samples"]},
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+
+
 def step_flop_counts(w, B=None, H=None):
     """Algorithmic forward and backward FLOPs of one step of workload w
     (visible pairs only for a block-sparse workload)."""
@@ -488,6 +621,8 @@ def step_flop_counts(w, B=None, H=None):
     H = w.H if H is None else H
     if w.nk:
         return perf.decode_flops(B, H, w.N, w.nk, w.d, w.causal), 0.0
+    if w.dtype == "e4m3":
+        return perf.fwd_flops(B, H, w.N, w.d, w.causal), 0.0
     m = workloads.block_mask(w)
     if m is not None:
         return (perf.fwd_flops_masked(B, H, w.N, w.d, w.causal, m),
@@ -503,6 +638,11 @@ def oracle_head_step(w, x, h):
         from oracle.decode import rect_forward
         rect_forward(x["q"][0, h], x["k"][0, h], x["v"][0, h], w.scale, w.causal)
         return
+    if w.dtype == "e4m3":
+        from oracle.fp8 import forward
+        forward(x["q8"][0, h], x["k8"][0, h], x["v8"][0, h], x["q_descale"], x["k_descale"],
+                x["v_descale"], w.scale, w.causal)
+        return
     qh, kh, vh, doh = (x[n][0, h] for n in ("q", "k", "v", "do"))
     m = workloads.block_mask(w)
     if m is not None:
@@ -517,7 +657,8 @@ def oracle_head_step(w, x, h):
 def cpu_baseline(w, seconds: float):
     """The fp64 oracle (as it stands) on a bounded sample of the workload:
     whole heads, forward and backward, until about ``seconds`` of CPU work."""
-    x = workloads.make_inputs(w, with_grad_out=True, B=1)
+    x = (workloads.make_fp8_inputs(w, B=1) if w.dtype == "e4m3"
+         else workloads.make_inputs(w, with_grad_out=True, B=1))
     cores = os.cpu_count() or 1
     n_heads, flops, t0 = 0, 0.0, time.perf_counter()
     per_head = sum(step_flop_counts(w, B=1, H=1))
@@ -529,7 +670,8 @@ def cpu_baseline(w, seconds: float):
             break
     el = time.perf_counter() - t0
     return {"value": round(flops / el / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{n_heads} head(s) of {w.name} (N={w.N}, d={w.d}), fwd+bwd, fp64 numpy "
+            "sample": f"{n_heads} head(s) of {w.name} (N={w.N}, d={w.d}), "
+                      f"{'fwd+bwd' if w.backward else 'fwd'}, fp64 numpy "
                       f"on the host ({el:.1f} s)"}
 
 
@@ -538,9 +680,14 @@ def run_reference(args):
     if rank != 0:
         return None
     w = workloads.WORKLOADS[args.workload]
-    x = (workloads.make_decode_inputs(w, B=1) if w.nk
-         else workloads.make_inputs(w, with_grad_out=True, B=1))
+    if w.nk:
+        x = workloads.make_decode_inputs(w, B=1)
+    elif w.dtype == "e4m3":
+        x = workloads.make_fp8_inputs(w, B=1)
+    else:
+        x = workloads.make_inputs(w, with_grad_out=True, B=1)
     per_head = sum(step_flop_counts(w, B=1, H=1))
+    passes = "fwd+bwd" if w.backward else "fwd"
 
     def step(i):
         oracle_head_step(w, x, i % w.H)
@@ -553,13 +700,13 @@ def run_reference(args):
     el = time.perf_counter() - t0
     value = per_head * args.steps / el / 1e12
     cores = os.cpu_count() or 1
-    sample = f"1 head of {w.name} (N={w.N}, d={w.d}) fwd+bwd per step, fp64 numpy oracle"
+    sample = f"1 head of {w.name} (N={w.N}, d={w.d}) {passes} per step, fp64 numpy oracle"
     return {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.describe(), "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                       "causal": w.causal, "passes": "fwd" if w.nk else "fwd+bwd"},
+                       "causal": w.causal, "passes": passes},
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
                              "kind": "oracle", "sample": sample},
@@ -639,6 +786,8 @@ def main(argv=None):
         return
     elif workloads.WORKLOADS[args.workload].nk:
         line = run_decode(args, peaks, kind)
+    elif workloads.WORKLOADS[args.workload].dtype == "e4m3":
+        line = run_fp8(args, peaks, kind)
     else:
         line = run_ours(args, peaks, kind)
     if line is not None:

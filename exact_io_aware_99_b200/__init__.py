@@ -8,7 +8,7 @@ Low-level entry points (same names as the C ABI): ``fa_forward``,
 ``fa_forward_ex``, ``fa_backward``, ``fa_backward_ex``,
 ``fa_backward_noalloc``, ``fa_forward_blocksparse``, ``fa_backward_blocksparse``,
 ``fa_forward_splitkv``, ``fa_splitkv_default_splits``, ``fa_splitkv_workspace_size``,
-``fa_backward_workspace_size``,
+``fa_backward_workspace_size``, ``fa_forward_fp8``, ``fa_quantize_fp8``,
 ``fa_status_string``, ``fa_device_status``, ``fa_set_wait_timeout_ns``,
 ``fa_selftest_wait_timeout``.
 
@@ -17,7 +17,10 @@ Convenience wrappers that allocate outputs with torch:
 -> (o, lse)`` and ``attention_backward(q, k, v, o, do, lse, scale=None,
 causal=False, block_mask=None) -> (dq, dk, dv)``, and
 ``attention_decode(q, k, v, scale=None, causal=False, num_splits=None)
--> (o, lse)`` for N_q queries against N_k keys (split-KV).
+-> (o, lse)`` for N_q queries against N_k keys (split-KV), and the FP8
+forward ``attention_forward_fp8(q8, k8, v8, q_descale, k_descale, v_descale,
+scale=None, causal=False) -> (o, lse)`` with ``quantize_fp8(x) -> (codes,
+descale)`` for its E4M3 inputs.
 
 The shared library is loaded on first use of any of these names (so the
 ``build`` submodule can run before it exists); using them without the built
@@ -31,9 +34,10 @@ _NATIVE = {
     "fa_backward_workspace_size", "fa_status_string", "fa_device_status",
     "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_forward_blocksparse",
     "fa_backward_blocksparse", "fa_forward_splitkv", "fa_splitkv_default_splits",
-    "fa_splitkv_workspace_size",
+    "fa_splitkv_workspace_size", "fa_forward_fp8", "fa_quantize_fp8",
 }
-_API = {"attention_forward", "attention_backward", "attention_decode"}
+_API = {"attention_forward", "attention_backward", "attention_decode",
+        "attention_forward_fp8", "quantize_fp8"}
 
 
 def __getattr__(name):

@@ -31,7 +31,8 @@ EXPORTS = (
     "fa_backward_ex", "fa_status_string", "fa_last_cuda_error", "fa_device_status",
     "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_backward_noalloc",
     "fa_forward_blocksparse", "fa_backward_blocksparse", "fa_forward_splitkv",
-    "fa_splitkv_default_splits", "fa_splitkv_workspace_size",
+    "fa_splitkv_default_splits", "fa_splitkv_workspace_size", "fa_forward_fp8",
+    "fa_quantize_fp8",
 )
 
 # Size of the library's built-in scratch array used by fa_backward_noalloc.
@@ -86,6 +87,10 @@ def _load() -> ctypes.CDLL:
     lib.fa_splitkv_workspace_size.argtypes = [I, I, I, I, I, I]
     lib.fa_splitkv_workspace_size.restype = S
     lib.fa_backward_noalloc.restype = I
+    lib.fa_forward_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, F, I, P]
+    lib.fa_forward_fp8.restype = I
+    lib.fa_quantize_fp8.argtypes = [P, I, S, P, P, P]
+    lib.fa_quantize_fp8.restype = I
     return lib
 
 
@@ -221,3 +226,21 @@ def fa_splitkv_default_splits(B, H, Nq, Nk) -> int:
 
 def fa_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits) -> int:
     return int(_lib.fa_splitkv_workspace_size(B, H, Nq, Nk, d, num_splits))
+
+
+def fa_forward_fp8(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, B, H, N, d, scale,
+                   causal, stream=None, check=True) -> int:
+    """FP8 forward: q8, k8, v8 are E4M3 codes (uint8 or float8_e4m3fn device
+    tensors), the descales device fp32 scalars or None (= 1)."""
+    st = _lib.fa_forward_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_descale), _ptr(k_descale),
+                             _ptr(v_descale), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                             int(bool(causal)), _stream(stream))
+    return _check(st, "fa_forward_fp8", check)
+
+
+def fa_quantize_fp8(x, dtype, n, codes, descale, stream=None, check=True) -> int:
+    """Per-tensor E4M3 quantisation of n elements of x (FA_BF16 or FA_FP32)
+    into codes (n bytes) and descale (one device fp32)."""
+    st = _lib.fa_quantize_fp8(_ptr(x), int(dtype), int(n), _ptr(codes), _ptr(descale),
+                              _stream(stream))
+    return _check(st, "fa_quantize_fp8", check)

@@ -109,3 +109,55 @@ def attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32)
     nat.fa_forward_splitkv(q, k, v, out, lse, B, H, Nq, Nk, d, scale, causal, s, ws, wbytes)
     return out, lse
+
+
+def _codes(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError("E4M3 inputs must be uint8 codes or float8_e4m3fn tensors")
+    return t
+
+
+def _descale(x, device) -> Optional[torch.Tensor]:
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        if not x.is_cuda or x.dtype != torch.float32 or x.numel() != 1:
+            raise ValueError("a descale tensor must be one fp32 element on the GPU")
+        return x
+    return torch.tensor([float(x)], device=device, dtype=torch.float32)
+
+
+def quantize_fp8(x: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-tensor E4M3 quantisation of a contiguous bf16 or fp32 CUDA tensor
+    (see ``fa_quantize_fp8``): returns the codes (uint8, x's shape) and the
+    descale factor (a one-element fp32 CUDA tensor, amax / 448)."""
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor")
+    codes = torch.empty(x.shape, device=x.device, dtype=torch.uint8)
+    descale = torch.empty(1, device=x.device, dtype=torch.float32)
+    nat.fa_quantize_fp8(x, _dtype_code(x), x.numel(), codes, descale)
+    return codes, descale
+
+
+def attention_forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor,
+                          q_descale=None, k_descale=None, v_descale=None,
+                          scale: Optional[float] = None, causal: bool = False,
+                          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None
+                          ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """FP8 forward (see ``fa_forward_fp8``): E4M3 q8, k8, v8 [B, H, N, d]
+    (uint8 codes or float8_e4m3fn), per-tensor descale factors (one-element
+    fp32 CUDA tensors, python floats, or None for 1).  Returns O (bf16) and
+    LSE (fp32)."""
+    for t in (q8, k8, v8):
+        _codes(t)
+        if not t.is_cuda or not t.is_contiguous() or t.shape != q8.shape:
+            raise ValueError("inputs must be contiguous CUDA tensors of one shape")
+    B, H, N, d = _dims(q8)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq, dk, dv = (_descale(x, q8.device) for x in (q_descale, k_descale, v_descale))
+    if out is None:
+        out = torch.empty((B, H, N, d), device=q8.device, dtype=torch.bfloat16)
+    if lse is None:
+        lse = torch.empty((B, H, N), device=q8.device, dtype=torch.float32)
+    nat.fa_forward_fp8(q8, k8, v8, dq, dk, dv, out, lse, B, H, N, d, scale, causal)
+    return out, lse

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_fp8.h"
 #include "fa_internal.h"
 
 namespace {
@@ -489,3 +490,77 @@ extern "C" fa_status fa_backward_noalloc(const void* q, const void* k, const voi
   return fa_backward_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, scratch,
                         static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES), FA_BF16, stream);
 }
+
+// ---------------------------------------------------------------------------
+// FP8 (E4M3) forward and the per-tensor E4M3 quantiser.
+namespace {
+
+// [BH, N, d] E4M3 (one byte per element) viewed as 3-D {d, N, BH}; box
+// {128, 128, 1}, a whole 128-byte swizzle row per query or key; columns past
+// d and rows past N read as zero.
+fa_status make_map_e4m3(CUtensorMap* m, const void* base, int BH, int N, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d)};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = static_cast<int>(r);
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_forward_fp8(const void* q, const void* k, const void* v, const float* q_descale,
+                         const float* k_descale, const float* v_descale, void* o, float* lse,
+                         int B, int H, int N, int d, float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, FA_BF16);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_MISALIGNED;
+  if ((q_descale && !aligned4(q_descale)) || (k_descale && !aligned4(k_descale)) ||
+      (v_descale && !aligned4(v_descale)))
+    return FA_ERR_MISALIGNED;
+  fa::Launch L;
+  st = device_context(stream, &L);
+  if (st != FA_OK) return st;
+  const int BH = B * H;
+  st = get_encoder();
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if ((st = make_map_e4m3(&tq, q, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map_e4m3(&tk, k, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map_e4m3(&tv, v, BH, N, d)) != FA_OK) return st;
+  cudaError_t e = fa::launch_fwd_fp8_sm100(tq, tk, tv, q_descale, k_descale, v_descale, o, lse,
+                                           BH, N, d, scale, causal ? 1 : 0, L);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+fa_status fa_quantize_fp8(const void* x, fa_dtype dtype, size_t n, void* codes, float* descale,
+                          void* stream) {
+  if (!x || !codes || !descale || n == 0) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP32) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(codes) || !aligned4(descale)) return FA_ERR_MISALIGNED;
+  fa::Launch L;
+  fa_status st = device_context(stream, &L);
+  if (st != FA_OK) return st;
+  cudaError_t e = cudaMemsetAsync(descale, 0, sizeof(float), L.stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = fa::launch_quantize_e4m3(x, dtype == FA_BF16 ? 1 : 0, n, static_cast<uint8_t*>(codes),
+                               descale, L);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+}  // extern "C"

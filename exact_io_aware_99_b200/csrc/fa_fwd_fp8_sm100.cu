@@ -1,0 +1,756 @@
+// fa_fwd_fp8_sm100.cu -- FP8 (E4M3) attention forward on B200 tensor cores
+// (tcgen05 kind::f8f6f4), and the per-tensor E4M3 quantiser.
+//
+// What it computes: the FlashAttention-2 forward (review page "FlashAttention-2:
+// Faster Attention with Better Parallelism and Work Partitioning", core-
+// algorithm answer, (1) tiling and (2) forward pass) with FP8 in both matmuls
+// and in the softmax's output, the extension the same page lists under
+// future work, (5) "FP8 and latest hardware", mixing FP8 with wider types as
+// its auto-tuning answer, 1 (2), asks:
+//   * Q, K, V are E4M3 with one fp32 dequantisation factor per tensor;
+//   * S = Q_i K_j^T runs as an E4M3 x E4M3 MMA with fp32 accumulation, and
+//     the Q and K factors fold into the exponent scale;
+//   * the softmax statistics (running max m, running sum l) stay fp32, and
+//     the probabilities P are rounded to E4M3 in tensor memory;
+//   * O += P V_j runs as an E4M3 x E4M3 MMA (P from tensor memory), fp32
+//     accumulation; the epilogue multiplies by v_descale / l and writes bf16
+//     O and the fp32 natural-log LSE.
+//
+// With the lazy rescaling threshold of 2^8 (the reference max moves only when
+// a row's max grows by more than 2^8), every probability is at most 2^8 = 256
+// and fits E4M3 (largest finite value 448) without a further scale; values
+// below 2^-6 of the reference max land in E4M3's subnormal range.
+//
+// Layout and schedule follow the bf16 forward (fa_fwd_sm100.cu): a work item
+// is a pair of 128-row query tiles of one head; warp 8 loads Q, K, V with TMA,
+// warp 9 issues the MMAs, warps 0-3 / 4-7 run the softmax of tile A / B; CTAs
+// take further items through cluster launch control, group-major and
+// longest-first.  What differs: an E4M3 row of up to 128 elements is one
+// 128-byte swizzle row, so every Q/K/V tile is a single 16 KB block (half the
+// bf16 tile) for any d <= 128; the S MMA runs ceil(d / 32) k-steps of 32
+// and the P V MMA four; P takes 32 TMEM columns (four E4M3 per column).
+#include <cuda_bf16.h>
+
+#include "fa_fp8.h"
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace fwd8 {
+
+constexpr int kBM = 128;              // query rows per tile (TMEM lanes)
+constexpr int kBN = 128;              // keys per K/V tile
+constexpr int kThreads = 384;
+// Registers per thread: 168 at launch (384 threads); the softmax warpgroups
+// then take kSoftmaxRegs each and the producer/MMA warpgroup keeps the rest:
+// 224 + 224 + 56 = 504 = 3 x 168, the launch budget of each lane slot.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 3 * kLaunchRegs - 2 * kSoftmaxRegs;
+static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kLaunchRegs, "register split over budget");
+constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold; keeps P <= 2^8
+#ifndef FA_FP8_POLY_EVERY
+#define FA_FP8_POLY_EVERY 0  // one column pair in this many uses the FMA-pipe exp2 (0: none)
+#endif
+constexpr int kPolyMod = FA_FP8_POLY_EVERY > 0 ? FA_FP8_POLY_EVERY : 1;
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+  static constexpr int TILE = kBM * 128;    // 128 rows x 128 bytes, one swizzle block
+  static constexpr int NST = 4;             // K and V ring stages
+  static constexpr int Q_OFF = 0;           // [2] tiles A, B
+  static constexpr int K_OFF = Q_OFF + 2 * TILE;
+  static constexpr int V_OFF = K_OFF + NST * TILE;
+  static constexpr int BAR_OFF = V_OFF + NST * TILE;
+  static constexpr int NBAR = 2 + 4 * NST + 6 + 4;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
+  static constexpr int SMEM = MISC_OFF + 48 + 1024;    // + slack for 1 KB alignment
+  static constexpr int KSTEPS = (D + 31) / 32;         // S MMA k-steps (32 E4M3 each)
+  static constexpr int NPV = (D + 15) / 16 * 16;       // P V MMA width (columns of O)
+  static_assert(D % 16 == 0 && D <= 128, "head dim must be a multiple of 16, <= 128");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(MISC_OFF % 16 == 0, "next-item responses need 16-byte alignment");
+};
+
+// ------------------------------------------------ kind::f8f6f4 primitives
+
+// Instruction descriptor of tcgen05.mma kind::f8f6f4: E4M3 A and B (format
+// code 0), fp32 D, shape M x N (x32), operand majors (0 = K, 1 = MN).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                              // D format f32
+         | (0u << 7)                            // A format E4M3
+         | (0u << 10)                           // B format E4M3
+         | (static_cast<uint32_t>(a_mn) << 15)
+         | (static_cast<uint32_t>(b_mn) << 16)
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, one 32-deep k-step of E4M3.
+__device__ __forceinline__ void mma_ss_e4m3(uint32_t d_tmem, SDesc a, SDesc b, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], A (K-major, four E4M3 per 32-bit column)
+// read from tensor memory.
+__device__ __forceinline__ void mma_ts_e4m3(uint32_t d_tmem, uint32_t a_tmem, SDesc b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Four floats to four E4M3 (round to nearest even, saturating to +-448):
+// a in bits 0-7, b in 8-15, c in 16-23, d in 24-31.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
+// Drain wait used only while aborting: ignores the abort flag, bounded by time.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(a, parity)) {
+    if (globaltimer_ns() - t0 > ctl.limit_ns) {
+      atomicCAS(ctl.status, 0, kSiteFp8Drain);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                         const WaitCtl& ctl, int site) {
+  const bool w = mbar_wait(bar, parity, abort, ctl, site);
+  return __all_sync(0xffffffffu, w);
+}
+
+// (bh, tile pair) and the key tiles each query tile of the pair visits (0
+// when tile B lies past N) for work item `idx`: `group` heads at a time
+// (their K and V stay in L2), longest tile pairs first, head fastest.
+template <bool CAUSAL>
+__device__ __forceinline__ void decode_item(int idx, int n_t, int BH, int group, int& bh,
+                                            int& pair, int (&n_x)[2]) {
+  const int n_pair = (n_t + 1) / 2;
+  const int per_group = group * n_pair;
+  const int g = idx / per_group;
+  const int r = idx - g * per_group;
+  const int gh = min(group, BH - g * group);
+  const int t = r / gh;
+  pair = n_pair - 1 - t;
+  bh = g * group + (r - t * gh);
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int qt = 2 * pair + x;
+    n_x[x] = qt >= n_t ? 0 : (CAUSAL ? min(qt + 1, n_t) : n_t);
+  }
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_descale,
+                   const float* __restrict__ k_descale, const float* __restrict__ v_descale,
+                   __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int N, int BH,
+                   int group, float scale_log2, WaitCtl ctl) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;         // Q tiles no longer read by the item's S MMAs
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + C::NST;
+  uint64_t* v_full = k_empty + C::NST;
+  uint64_t* v_empty = v_full + C::NST;
+  uint64_t* s_full = v_empty + C::NST;  // [2] per tile
+  uint64_t* p_full = s_full + 2;        // [2] per tile
+  uint64_t* o_done = p_full + 2;        // [2] per tile
+  uint64_t* nxt_full = o_done + 2;      // [2] next-item responses
+  uint64_t* nxt_empty = nxt_full + 2;   // [2]
+  uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 36);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int n_t = (N + kBN - 1) / kBN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_full + x, kBM);
+      mbar_init(o_done + x, 1);
+      mbar_init(nxt_full + x, 1);
+      mbar_init(nxt_empty + x, 9);  // MMA warp + 8 softmax warps
+    }
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Work item i of this CTA: its own index first, then the CTAs it
+  // cancelled (the producer's request during item i - 1, slot i & 1).
+  auto next_item = [&](int i, int& idx, int site) -> bool {
+    if (i == 0) {
+      idx = static_cast<int>(blockIdx.x);
+      return true;
+    }
+    const int sl = i & 1;
+    if (!wait_all(nxt_full + sl, static_cast<uint32_t>((i - 1) >> 1) & 1, abort, ctl, site))
+      return false;
+    idx = clc_result_x(nxt_resp + 16 * sl);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(nxt_empty + sl);
+    return true;
+  };
+
+  if (warp >= 8) {
+  regs_decrease<kControlRegs>();
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      auto wait = [&](uint64_t* bar, uint32_t par) -> bool {
+        return mbar_wait(bar, par, abort, ctl, kSiteFp8Producer);
+      };
+      int last_k[C::NST], last_v[C::NST];
+#pragma unroll
+      for (int s = 0; s < C::NST; ++s) last_k[s] = last_v[s] = -1;
+      int q_issued = 0;
+      int nxt_pending = -1;
+      uint32_t nxt_pending_par = 0;
+      uint32_t kv = 0;  // K/V ring uses so far
+      int idx = static_cast<int>(blockIdx.x);
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        if (i > 0) {
+          const int sl = i & 1;
+          if (!wait(nxt_full + sl, static_cast<uint32_t>((i - 1) >> 1) & 1)) break;
+          nxt_pending = -1;
+          idx = clc_result_x(nxt_resp + 16 * sl);
+          if (idx < 0) break;
+        }
+        int bh, pair, n_x[2];
+        decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+        const int n_max = max(n_x[0], n_x[1]);
+        // Q of this item replaces the previous item's once its S MMAs are done.
+        if (q_issued > 0 && !wait(q_empty, static_cast<uint32_t>(q_issued - 1) & 1)) break;
+        const int nq = n_x[1] > 0 ? 2 : 1;
+        mbar_arrive_expect_tx(q_full, nq * C::TILE);
+        for (int x = 0; x < nq; ++x)
+          tma_load_3d(&tm_q, q_full, smem + C::Q_OFF + x * C::TILE, 0, (2 * pair + x) * kBM, bh);
+        ++q_issued;
+        for (int j = 0; j < n_max; ++j, ++kv) {
+          const int s = static_cast<int>(kv % C::NST);
+          const uint32_t u = kv / C::NST;
+          if (kv >= C::NST && !wait(k_empty + s, (u - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(k_full + s, C::TILE);
+          tma_load_3d(&tm_k, k_full + s, smem + C::K_OFF + s * C::TILE, 0, j * kBN, bh);
+          last_k[s] = static_cast<int>(u);
+          if (kv >= C::NST && !wait(v_empty + s, (u - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(v_full + s, C::TILE);
+          tma_load_3d(&tm_v, v_full + s, smem + C::V_OFF + s * C::TILE, 0, j * kBN, bh);
+          last_v[s] = static_cast<int>(u);
+        }
+        if (!ok) break;
+        // Ask for the next item now, while this one's MMAs and softmax run.
+        const int sl1 = (i + 1) & 1;
+        const uint32_t u1 = static_cast<uint32_t>(i >> 1);
+        if (u1 > 0 && !wait(nxt_empty + sl1, (u1 - 1) & 1)) break;
+        mbar_arrive_expect_tx(nxt_full + sl1, 16);
+        clc_try_cancel(nxt_resp + 16 * sl1, nxt_full + sl1);
+        nxt_pending = sl1;
+        nxt_pending_par = u1 & 1;
+      }
+      if (*abort) {
+        // Let every copy and request this CTA started land before shared
+        // memory is released.
+        if (q_issued > 0) drain_wait(q_full, static_cast<uint32_t>(q_issued - 1) & 1, ctl);
+        for (int s = 0; s < C::NST; ++s) {
+          if (last_k[s] >= 0) drain_wait(k_full + s, last_k[s] & 1, ctl);
+          if (last_v[s] >= 0) drain_wait(v_full + s, last_v[s] & 1, ctl);
+        }
+        if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    // The whole warp runs the schedule; the elected lane issues and commits.
+    const bool leader = elect_one();
+    constexpr uint32_t kIdescS = idesc_e4m3(kBM, kBN, 0, 0);
+    constexpr uint32_t kIdescPV = idesc_e4m3(kBM, C::NPV, 0, 1);
+    const SDesc q_desc = sdesc(sbase + C::Q_OFF, 16, 1024);        // K-major
+    const SDesc k_desc = sdesc(sbase + C::K_OFF, 16, 1024);        // K-major
+    const SDesc v_desc = sdesc(sbase + C::V_OFF, C::TILE, 1024);   // MN-major, one atom wide
+    uint32_t kv_base = 0;
+    uint32_t p_base[2] = {0u, 0u};
+    int k_seen = -1;
+    auto wait_k = [&](int r) -> bool {
+      if (r <= k_seen) return true;
+      if (!wait_all(k_full + r % C::NST, static_cast<uint32_t>(r / C::NST) & 1, abort, ctl,
+                    kSiteFp8Mma))
+        return false;
+      k_seen = r;
+      tc_fence_after();
+      return true;
+    };
+    auto issue_s = [&](int x, int r) {  // S_x = Q_x K^T, K in ring use r
+      if (leader) {
+        const SDesc qd = q_desc + x * C::TILE;
+        const SDesc kd = k_desc + (r % C::NST) * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS; ++kk)
+          mma_ss_e4m3(tmem + x * kBN, qd + kk * 32, kd + kk * 32, kIdescS, kk > 0 ? 1u : 0u);
+        mma_commit(s_full + x);
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int x, int r, bool first) {  // O_x (+)= P_x V, P_x from TMEM
+      if (leader) {
+        const SDesc vd = v_desc + (r % C::NST) * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 32; ++kk)
+          mma_ts_e4m3(tmem + 256 + x * kBN, tmem + x * kBN + kk * 8, vd + kk * 32 * 128,
+                      kIdescPV, (!first || kk > 0) ? 1u : 0u);
+        mma_commit(o_done + x);
+      }
+      __syncwarp();
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (leader) mma_commit(bar);
+      __syncwarp();
+    };
+    bool ok = true;
+    int idx = 0;
+    uint32_t q_items = 0;
+    for (int i = 0; ok; ++i) {
+      if (!next_item(i, idx, kSiteFp8Mma)) break;
+      if (idx < 0) break;
+      int bh, pair, n_x[2];
+      decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+      const int n_max = max(n_x[0], n_x[1]);
+      const int r0 = static_cast<int>(kv_base);
+      ok = wait_all(q_full, q_items & 1, abort, ctl, kSiteFp8Mma) && wait_k(r0);
+      ++q_items;
+      if (!ok) break;
+      tc_fence_after();
+      for (int x = 0; x < 2; ++x)
+        if (n_x[x] > 0) issue_s(x, r0);
+      commit(k_empty + r0 % C::NST);
+      if (n_max == 1) commit(q_empty);
+      for (int j = 0; ok && j < n_max; ++j) {
+        const int r = r0 + j;
+        if (!wait_all(v_full + r % C::NST, static_cast<uint32_t>(r / C::NST) & 1, abort, ctl,
+                      kSiteFp8Mma)) {
+          ok = false;
+          break;
+        }
+        for (int x = 0; ok && x < 2; ++x) {
+          if (j >= n_x[x]) continue;
+          if (!wait_all(p_full + x, (p_base[x] + j) & 1, abort, ctl, kSiteFp8Mma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(x, r, j == 0);
+          if (j + 1 < n_x[x]) {
+            if (!wait_k(r + 1)) {
+              ok = false;
+              break;
+            }
+            issue_s(x, r + 1);
+          }
+        }
+        if (!ok) break;
+        commit(v_empty + r % C::NST);
+        if (j + 1 < n_max) commit(k_empty + (r + 1) % C::NST);
+        if (j + 2 == n_max) commit(q_empty);  // the item's last S MMAs are issued
+      }
+      kv_base += static_cast<uint32_t>(n_max);
+      p_base[0] += static_cast<uint32_t>(n_x[0]);
+      p_base[1] += static_cast<uint32_t>(n_x[1]);
+    }
+    __syncwarp();
+  }
+  } else {
+    regs_increase<kSoftmaxRegs>();
+    // --------------------------------------- softmax (warps 0-3: A, 4-7: B)
+    const int x = warp >> 2;
+    const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t col_s = x * kBN;
+    const uint32_t col_o = 256 + x * kBN;
+    // The Q and K factors scale every score, V's every output.
+    const float dqk = (q_descale ? *q_descale : 1.f) * (k_descale ? *k_descale : 1.f);
+    const float dv = v_descale ? *v_descale : 1.f;
+    const float sl2 = scale_log2 * dqk;
+    uint32_t s_base = 0;  // s_full / o_done phases of this tile before the current item
+    bool ok = true;
+    int idx = 0;
+    for (int i = 0; ok; ++i) {
+      if (!next_item(i, idx, kSiteFp8Softmax)) break;
+      if (idx < 0) break;
+      int bh, pair, n_x[2];
+      decode_item<CAUSAL>(idx, n_t, BH, group, bh, pair, n_x);
+      const int n_kv = n_x[x];
+      if (n_kv == 0) continue;  // tile past N
+      const int qt_x = 2 * pair + x;
+      const int q_idx = qt_x * kBM + r;
+      float m = -INFINITY;  // reference max, base-2 scaled units
+      float l = 0.f;
+      for (int j = 0; j < n_kv; ++j) {
+        if (!wait_all(s_full + x, (s_base + j) & 1, abort, ctl, kSiteFp8Softmax)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[kBN];
+        {
+          uint32_t t0[32], t1[32];
+          tmem_ld32(lane_base + col_s + 0, t0);
+          tmem_ld32(lane_base + col_s + 32, t1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            s[c] = __uint_as_float(t0[c]);
+            s[32 + c] = __uint_as_float(t1[c]);
+          }
+          tmem_ld32(lane_base + col_s + 64, t0);
+          tmem_ld32(lane_base + col_s + 96, t1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            s[64 + c] = __uint_as_float(t0[c]);
+            s[96 + c] = __uint_as_float(t1[c]);
+          }
+        }
+        const int kv0 = j * kBN;
+        const bool masked = (CAUSAL && j == n_kv - 1) || kv0 + kBN > N;
+        const int lim = masked ? min(N - kv0, CAUSAL ? (q_idx - kv0 + 1) : kBN) : kBN;
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
+        float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+        for (int c = 4; c < kBN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float m_cand = fmaxf(m, mx * sl2);
+        const bool grow = m_cand > m + kRescaleLog2;  // true on the first tile
+        const float alpha = grow ? ex2(m - m_cand) : 1.f;
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O_x += P_x(j-1) V completed before S_x(j) (same issuing thread,
+          // in order), so O_x can be rescaled now.
+#pragma unroll
+          for (int c = 0; c < C::NPV / 16; ++c) {
+            uint32_t o16[16];
+            tmem_ld16(lane_base + col_o + c * 16, o16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
+            tmem_st16(lane_base + col_o + c * 16, o16);
+          }
+        }
+        if (grow) {
+          l *= alpha;
+          m = m_cand;
+        }
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        const float2 sc2 = make_float2(sl2, sl2);
+        const float2 nm2 = make_float2(neg_m, neg_m);
+        float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+        uint32_t pk[kBN / 4];
+#pragma unroll
+        for (int c = 0; c < kBN / 4; ++c) {
+          float2 p2[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int e = 2 * (2 * c + h);
+            const float2 xx = __ffma2_rn(make_float2(s[e], s[e + 1]), sc2, nm2);
+            float2 p;
+            if (FA_FP8_POLY_EVERY > 0 && (2 * c + h) % kPolyMod == kPolyMod - 1) {
+              p = exp2_fma2(xx);
+              if (masked) {
+                if (e >= lim) p.x = 0.f;
+                if (e + 1 >= lim) p.y = 0.f;
+              }
+            } else {
+              p = make_float2(ex2(xx.x), ex2(xx.y));
+            }
+            rs2[(2 * c + h) & 3] = __fadd2_rn(rs2[(2 * c + h) & 3], p);
+            p2[h] = p;
+          }
+          pk[c] = pack_e4m3x4(p2[0].x, p2[0].y, p2[1].x, p2[1].y);
+        }
+        const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+        l += rsa.x + rsa.y;
+        tmem_st32(lane_base + col_s, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + x);
+      }
+      // -------------------------------------------------------- epilogue
+      if (ok && wait_all(o_done + x, (s_base + n_kv - 1) & 1, abort, ctl, kSiteFp8Epilogue)) {
+        tc_fence_after();
+        const float f = dv / l;  // l >= 1: the row's reference max contributes 2^0
+        const bool valid = q_idx < N;
+        const float lse_row = (m + __log2f(l)) * 0.69314718055994531f;
+        uint32_t* orow = reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
+#pragma unroll
+        for (int c = 0; c < C::NPV / 16; ++c) {
+          uint32_t o16[16];
+          tmem_ld16(lane_base + col_o + c * 16, o16);
+          tmem_wait_ld();
+          uint32_t pkd[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            pkd[e] = pack_bf16(__uint_as_float(o16[2 * e]) * f, __uint_as_float(o16[2 * e + 1]) * f);
+          if (valid) {
+            // D is a multiple of 16, so 16-column chunks never straddle it.
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 8);
+            dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+            dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+          }
+        }
+        if (valid) lse[static_cast<size_t>(bh) * N + q_idx] = lse_row;
+        // The next item's first P V (accumulate off) overwrites O_x only
+        // after this warpgroup's next P, so the loads above are complete.
+        tc_fence_before();
+      } else {
+        ok = false;
+      }
+      s_base += static_cast<uint32_t>(n_kv);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const float* q_descale, const float* k_descale, const float* v_descale,
+                   void* o, float* lse, int BH, int N, float scale, const Launch& L) {
+  using C = Cfg<D>;
+  static bool configured = false;
+  if (!configured) {
+    // The register split assumes exactly kLaunchRegs per thread at launch;
+    // with fewer, the softmax warps' increase would wait forever.
+    cudaFuncAttributes fattr;
+    cudaError_t e = cudaFuncGetAttributes(&fattr, fwd_fp8_kernel<D, CAUSAL>);
+    if (e != cudaSuccess) return e;
+    if (fattr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(fwd_fp8_kernel<D, CAUSAL>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int n_t = (N + kBM - 1) / kBM;
+  const int n_pair = (n_t + 1) / 2;
+  // Heads per group: K and V of a head (2 N d bytes in E4M3) are what every
+  // item of the head re-reads; a group's share stays within the L2 budget.
+  const long long per_head = 2LL * N * D;
+  int group = static_cast<int>(l2_group_bytes(CAUSAL) / (per_head > 0 ? per_head : 1));
+  group = group < 1 ? 1 : (group > BH ? BH : group);
+  const long long blocks = static_cast<long long>(BH) * n_pair;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  WaitCtl ctl{L.status, L.limit_ns};
+  fwd_fp8_kernel<D, CAUSAL><<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
+      tq, tk, tv, q_descale, k_descale, v_descale, static_cast<__nv_bfloat16*>(o), lse, N, BH,
+      group, scale_log2, ctl);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const float* dq, const float* dk, const float* dv, void* o, float* lse,
+                     int BH, int N, float scale, int causal, const Launch& L) {
+  return causal ? launch<D, true>(tq, tk, tv, dq, dk, dv, o, lse, BH, N, scale, L)
+                : launch<D, false>(tq, tk, tv, dq, dk, dv, o, lse, BH, N, scale, L);
+}
+
+// ------------------------------------------------- per-tensor quantiser
+
+constexpr int kQThreads = 256;
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) {
+  return v;
+}
+
+// amax = max |x| over n elements, as the bits of a non-negative float
+// (ordered like unsigned integers), merged into *amax_bits with atomicMax.
+template <typename T>
+__global__ void __launch_bounds__(kQThreads) amax_kernel(const T* __restrict__ x, size_t n,
+                                                         unsigned* amax_bits) {
+  constexpr int V = 16 / sizeof(T);  // elements per 16-byte load
+  const size_t nv = n / V;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  const size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  unsigned m = 0u;
+  const uint4* xv = reinterpret_cast<const uint4*>(x);
+  for (size_t i = t; i < nv; i += stride) {
+    const uint4 u = __ldg(xv + i);
+    const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+    for (int k = 0; k < V; ++k) m = max(m, __float_as_uint(fabsf(to_f32<T>(e[k]))));
+  }
+  for (size_t i = nv * V + t; i < n; i += stride) m = max(m, __float_as_uint(fabsf(to_f32<T>(x[i]))));
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(amax_bits, m);
+}
+
+// codes = RN_satfinite(x * (448 / amax)); the quotient and the product are
+// single fp32 operations rounded to nearest.
+template <typename T>
+__global__ void __launch_bounds__(kQThreads) quantize_kernel(const T* __restrict__ x, size_t n,
+                                                             const unsigned* amax_bits,
+                                                             uint8_t* __restrict__ codes) {
+  const float amax = __uint_as_float(*amax_bits);
+  const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+  const size_t nv = n / 8;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  const size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (size_t i = t; i < nv; i += stride) {
+    float f[8];
+    if (sizeof(T) == 2) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(x) + i);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) f[k] = __fmul_rn(to_f32<T>(e[k]), inv);
+    } else {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(x) + 2 * i);
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(x) + 2 * i + 1);
+      const float* ea = reinterpret_cast<const float*>(&a);
+      const float* eb = reinterpret_cast<const float*>(&b);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        f[k] = __fmul_rn(ea[k], inv);
+        f[4 + k] = __fmul_rn(eb[k], inv);
+      }
+    }
+    reinterpret_cast<uint2*>(codes)[i] =
+        make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
+  }
+  for (size_t i = nv * 8 + t; i < n; i += stride)
+    codes[i] = static_cast<uint8_t>(pack_e4m3x4(__fmul_rn(to_f32<T>(x[i]), inv), 0.f, 0.f, 0.f) &
+                                    0xFFu);
+}
+
+__global__ void descale_kernel(float* descale) {
+  const float amax = *descale;  // holds amax's bits until now
+  *descale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+}
+
+template <typename T>
+cudaError_t launch_quantize(const T* x, size_t n, uint8_t* codes, float* descale,
+                            const Launch& L) {
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t want = (n / 8 + kQThreads - 1) / kQThreads;
+  const unsigned blocks =
+      static_cast<unsigned>(want < 1 ? 1 : (want > static_cast<size_t>(sms) * 8 ? sms * 8 : want));
+  unsigned* bits = reinterpret_cast<unsigned*>(descale);
+  amax_kernel<T><<<blocks, kQThreads, 0, L.stream>>>(x, n, bits);
+  quantize_kernel<T><<<blocks, kQThreads, 0, L.stream>>>(x, n, bits, codes);
+  descale_kernel<<<1, 1, 0, L.stream>>>(descale);
+  return cudaGetLastError();
+}
+
+}  // namespace fwd8
+}  // namespace fa
+
+namespace fa {
+
+cudaError_t launch_fwd_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const float* q_descale,
+                                 const float* k_descale, const float* v_descale, void* o,
+                                 float* lse, int BH, int N, int d, float scale, int causal,
+                                 const Launch& L) {
+  switch (d) {
+    case 64:
+      return fwd8::launch_d<64>(tq, tk, tv, q_descale, k_descale, v_descale, o, lse, BH, N,
+                                scale, causal, L);
+    case 80:
+      return fwd8::launch_d<80>(tq, tk, tv, q_descale, k_descale, v_descale, o, lse, BH, N,
+                                scale, causal, L);
+    case 128:
+      return fwd8::launch_d<128>(tq, tk, tv, q_descale, k_descale, v_descale, o, lse, BH, N,
+                                 scale, causal, L);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_quantize_e4m3(const void* x, int is_bf16, size_t n, uint8_t* codes,
+                                 float* descale, const Launch& L) {
+  return is_bf16 ? fwd8::launch_quantize(static_cast<const __nv_bfloat16*>(x), n, codes,
+                                         descale, L)
+                 : fwd8::launch_quantize(static_cast<const float*>(x), n, codes, descale, L);
+}
+
+}  // namespace fa

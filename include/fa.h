@@ -252,6 +252,54 @@ FA_API fa_status fa_backward_noalloc(const void* q, const void* k, const void* v
                               int B, int H, int N, int d, float scale, int causal,
                               void* stream);
 
+/*
+ * fa_forward_fp8 -- FP8 forward: the attention of fa_forward computed with
+ * E4M3 inputs and E4M3 tensor-core matmuls, the extension the
+ * "FlashAttention-2: Faster Attention with Better Parallelism and Work
+ * Partitioning" review page lists under future work, (5) "FP8 and latest
+ * hardware" (FP8 in the matmuls and the softmax), mixed with wider types
+ * where accuracy needs them (its auto-tuning answer, section 1 (2)).
+ *   q, k, v     E4M3 codes (1 byte each: sign, 4 exponent bits with bias 7,
+ *               3 mantissa bits; 0x7F / 0xFF are NaN), [B, H, N, d]
+ *               contiguous, 16-byte aligned.
+ *   q_descale, k_descale, v_descale
+ *               device pointers to one fp32 dequantisation factor each
+ *               (element = value(code) * descale); NULL means 1.  Read by
+ *               the kernel, so they may be produced on the device (e.g. by
+ *               fa_quantize_fp8) without a host synchronisation.
+ *   o           bf16 [B, H, N, d]; lse fp32 [B, H, N] (natural log).
+ * Both products Q K^T and P V run as E4M3 x E4M3 with fp32 accumulation; the
+ * softmax statistics are fp32 and the probabilities are rounded to E4M3
+ * (relative error <= 2^-4 each) before P V.  The result approximates the
+ * exact attention of the dequantised inputs; the rounding of P bounds the
+ * difference per element.  d in {64, 80, 128}; scale, causal, stream and
+ * errors as fa_forward.
+ */
+FA_API fa_status fa_forward_fp8(const void* q, const void* k, const void* v,
+                                const float* q_descale, const float* k_descale,
+                                const float* v_descale, void* o, float* lse,
+                                int B, int H, int N, int d, float scale, int causal,
+                                void* stream);
+
+/*
+ * fa_quantize_fp8 -- per-tensor E4M3 quantisation for fa_forward_fp8's
+ * inputs (the pages fix no FP8 scaling; this is the plain per-tensor
+ * reading): amax = max |x| over the n elements, codes[e] =
+ * RN(x[e] * (448 / amax)) with saturation to +-448, *descale = amax / 448
+ * (each quotient and product one fp32 operation rounded to nearest; amax = 0
+ * gives codes 0 and descale 1).
+ *   x        device pointer, n elements of dtype FA_BF16 or FA_FP32,
+ *            16-byte aligned.
+ *   codes    device pointer, n bytes, 16-byte aligned.
+ *   descale  device pointer to one fp32 (4-byte aligned); written on the
+ *            stream, so a following fa_forward_fp8 on the same stream can
+ *            read it.
+ * Non-finite inputs give unspecified codes.  n = 0 or a null pointer is
+ * FA_ERR_INVALID_ARG.
+ */
+FA_API fa_status fa_quantize_fp8(const void* x, fa_dtype dtype, size_t n, void* codes,
+                                 float* descale, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_API const char* fa_status_string(fa_status s);
 

@@ -212,3 +212,41 @@ def test_decode_flop_and_byte_counts():
     assert perf.decode_pairs(300, 300, True) == 300 * 301 / 2
     assert perf.decode_flops(2, 3, 4, 9, 16, False) == 4 * 16 * 2 * 3 * 36
     assert perf.decode_bytes(1, 1, 2, 10, 8) == 2 * 2 * 8 * 2 + 2 * 10 * 8 * 2 + 4 * 2
+
+
+def test_fp8_entry_points_reject_bad_arguments_before_any_device_call():
+    fa = _lib()
+    # null input, unsupported head dim, misaligned code or descale pointers
+    st = fa.fa_forward_fp8(0, A, A, None, None, None, A, A, 1, 1, 128, 64, 0.1, 0,
+                           stream=0, check=False)
+    assert st == -1
+    st = fa.fa_forward_fp8(A, A, A, None, None, None, A, A, 1, 1, 128, 96, 0.1, 0,
+                           stream=0, check=False)
+    assert st == -2
+    st = fa.fa_forward_fp8(A + 8, A, A, None, None, None, A, A, 1, 1, 128, 64, 0.1, 0,
+                           stream=0, check=False)
+    assert st == -3
+    st = fa.fa_forward_fp8(A, A, A, A + 2, None, None, A, A, 1, 1, 128, 64, 0.1, 0,
+                           stream=0, check=False)
+    assert st == -3
+    st = fa.fa_forward_fp8(A, A, A, None, None, None, A, A, 1, 1, 0, 64, 0.1, 0,
+                           stream=0, check=False)
+    assert st == -1
+    # quantiser: empty input, unknown dtype, misaligned codes
+    assert fa.fa_quantize_fp8(A, fa.FA_BF16, 0, A, A, stream=0, check=False) == -1
+    assert fa.fa_quantize_fp8(A, 9, 16, A, A, stream=0, check=False) == -2
+    assert fa.fa_quantize_fp8(A, fa.FA_FP32, 16, A + 4, A, stream=0, check=False) == -3
+
+
+def test_fp8_workload_and_generators():
+    import torch
+    w = workloads.WORKLOADS["fp8_causal_d128"]
+    assert (w.B, w.H, w.N, w.d, w.dtype, w.causal, w.backward) == \
+        (4, 16, 4096, 128, "e4m3", True, False)
+    a = workloads.make_fp8_inputs(w, B=1, H=1, N=64)
+    b = workloads.make_fp8_inputs(w, B=1, H=1, N=64)
+    assert a["q8"].dtype == torch.uint8 and a["q8"].shape == (1, 1, 64, 128)
+    assert torch.equal(a["k8"], b["k8"]) and a["v_descale"] == b["v_descale"]
+    # the largest magnitude of each tensor maps onto 448 (code 0x7E / 0xFE)
+    for n in ("q8", "k8", "v8"):
+        assert int((a[n] & 0x7F).max()) == 0x7E
