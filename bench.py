@@ -65,6 +65,23 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(x: float, ws: int, device) -> float:
+    """The largest x over all ranks (for a time: the slowest rank's), x itself
+    on one rank.  Every rank must call it at the same point."""
+    if ws <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(ws: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job TFLOP/s: every rank does flops_per_rank in ms (the
+    max over ranks), so the job does ws times that."""
+    return ws * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -243,16 +260,12 @@ def run_ours(args, peaks, peak_kind):
     st, site = fa.fa_device_status(reset=True)
     if st != 0:
         raise RuntimeError(f"device wait timed out (site {site:#x})")
-    if ws > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, ws, dev)
     ms_step = total_ms / args.steps
 
     flops_f, flops_b = step_flop_counts(w)
     step_flops = flops_f + flops_b
-    value = ws * step_flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(ws, step_flops, ms_step)
 
     # End to end through the public API with host buffers: pinned host inputs
     # copied in, both passes, outputs copied back, every step.
@@ -288,13 +301,8 @@ def run_ours(args, peaks, peak_kind):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = a.elapsed_time(b) / ne
-        if ws > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": round(ws * step_flops / (e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+        e_ms = max_over_ranks(a.elapsed_time(b) / ne, ws, dev)
+        e2e = {"value": round(whole_job_tflops(ws, step_flops, e_ms), 3), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e_ms, 4)}
 
     cpu = None
@@ -397,14 +405,10 @@ def run_decode(args, peaks, peak_kind):
     if st != 0:
         raise RuntimeError(f"device wait timed out (site {site:#x})")
     ms = a.elapsed_time(b) / args.steps
-    if ws > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, ws, dev)
     flops = perf.decode_flops(B, H, Nq, Nk, d, w.causal)
     nbytes = perf.decode_bytes(B, H, Nq, Nk, d)
-    value = ws * flops / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(ws, flops, ms)
     gbs = nbytes / (ms * 1e-3) / 1e9
 
     e2e = None
@@ -433,8 +437,8 @@ def run_decode(args, peaks, peak_kind):
             e2e_step()
         eb.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = ea.elapsed_time(eb) / ne
-        e2e = {"value": round(ws * flops / (e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+        e_ms = max_over_ranks(ea.elapsed_time(eb) / ne, ws, dev)
+        e2e = {"value": round(whole_job_tflops(ws, flops, e_ms), 3), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e_ms, 4)}
 
     cpu = None
@@ -539,13 +543,9 @@ def run_fp8(args, peaks, peak_kind):
     if st != 0:
         raise RuntimeError(f"device wait timed out (site {site:#x})")
     ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    if ws > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, ws, dev)
     flops = perf.fwd_flops(B, H, N, d, w.causal)
-    value = ws * flops / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(ws, flops, ms)
 
     e2e = None
     if not args.no_e2e:
@@ -573,8 +573,8 @@ def run_fp8(args, peaks, peak_kind):
             e2e_step()
         eb.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = ea.elapsed_time(eb) / ne
-        e2e = {"value": round(ws * flops / (e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+        e_ms = max_over_ranks(ea.elapsed_time(eb) / ne, ws, dev)
+        e2e = {"value": round(whole_job_tflops(ws, flops, e_ms), 3), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e_ms, 4)}
 
     cpu = None
