@@ -80,3 +80,25 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
+
+
+def test_reference_arm_json_contract_on_one_rank():
+    # one short step per workload kind (dense, FP8, decode); keys of the line
+    for wl in ("fp32_small", "fp8_causal_d128", "decode_d128"):
+        r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", wl,
+                            "--steps", "1", "--warmup", "0"], cwd=ROOT, capture_output=True,
+                           text=True, timeout=300)
+        assert r.returncode == 0, r.stderr[-2000:]
+        lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+        assert len(lines) == 1
+        line = json.loads(lines[0])
+        for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                    "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                    "impl", "cpu_baseline", "e2e"):
+            assert key in line, (wl, key)
+        assert line["impl"] == "reference" and line["n_gpus"] == 1
+        assert line["config"]["workload"].startswith(wl)
+        assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
+                               "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+        assert line["cpu_baseline"]["value"] == line["value"]
+        assert line["cpu_baseline"]["cores"] >= 1
