@@ -36,7 +36,9 @@
  *   Pointers   device pointers, each 16-byte aligned; the caller owns all
  *              memory.  The library never allocates device memory.  It keeps
  *              one 4-byte device status word per process (a file-scope
- *              device variable) and nothing else.
+ *              device variable) and the fixed scratch array of
+ *              fa_backward_noalloc (FA_NOALLOC_SCRATCH_BYTES, also
+ *              file-scope), nothing else.
  *   Streams    `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *              default stream).  Every call is asynchronous on that stream;
  *              no call synchronises the host except fa_device_status.
