@@ -250,3 +250,12 @@ def test_fp8_workload_and_generators():
     # the largest magnitude of each tensor maps onto 448 (code 0x7E / 0xFE)
     for n in ("q8", "k8", "v8"):
         assert int((a[n] & 0x7F).max()) == 0x7E
+
+
+def test_fp8_step_counts_only_the_forward():
+    import bench
+    w = workloads.WORKLOADS["fp8_causal_d128"]
+    f, b = bench.step_flop_counts(w)
+    assert b == 0.0
+    assert f == perf.fwd_flops(4, 16, 4096, 128, True)
+    assert abs(f - 274.9e9) < 0.1e9
