@@ -706,7 +706,10 @@ def run_reference(args):
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.describe(), "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                       "causal": w.causal, "passes": passes},
+                       "causal": w.causal, "passes": passes,
+                       "timed_per_step": {"B": 1, "H": 1, "N": w.N, "d": w.d,
+                                          "note": "one head of the workload per step "
+                                                  "(heads cycle); value = its FLOPs / time"}},
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
                              "kind": "oracle", "sample": sample},

@@ -24,8 +24,11 @@ std::atomic<unsigned long long> g_limit_ns{kDefaultLimitNs};
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
+// Filled in once per device under g_dev_mu; `checked` is published with a
+// release store after `status`, so a thread that reads it with acquire and
+// sees 1 also sees the status address.
 struct DeviceInfo {
-  int checked = 0;  // 0 unknown, 1 supported, -1 unsupported
+  std::atomic<int> checked{0};  // 0 unknown, 1 supported, -1 unsupported
   int* status = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -51,24 +54,27 @@ fa_status device_context(void* stream, fa::Launch* L) {
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
   DeviceInfo& di = g_dev[dev];
-  if (di.checked == 0) {
+  int checked = di.checked.load(std::memory_order_acquire);
+  if (checked == 0) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (di.checked == 0) {
+    checked = di.checked.load(std::memory_order_relaxed);
+    if (checked == 0) {
       cudaDeviceProp prop;
       e = cudaGetDeviceProperties(&prop, dev);
       if (e != cudaSuccess) return cuda_fail(e);
       if (prop.major != 10 || prop.minor != 0) {
-        di.checked = -1;
+        checked = -1;
       } else {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_fa_status);
         if (e != cudaSuccess) return cuda_fail(e);
         di.status = static_cast<int*>(p);
-        di.checked = 1;
+        checked = 1;
       }
+      di.checked.store(checked, std::memory_order_release);
     }
   }
-  if (di.checked < 0) return FA_ERR_UNSUPPORTED;
+  if (checked < 0) return FA_ERR_UNSUPPORTED;
   L->stream = static_cast<cudaStream_t>(stream);
   L->status = di.status;
   L->limit_ns = g_limit_ns.load(std::memory_order_relaxed);
@@ -443,35 +449,38 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
 //
 // The array lives in device memory of every GPU that loads the library, for
 // the life of the process.  All calls on a GPU share it and it keeps the
-// previous call's contents; the backward's preprocess kernel clears the dQ
-// accumulator and rewrites the row vectors on every call, so nothing carries
-// over between calls, but two calls whose kernels overlap on the GPU (for
+// previous call's contents.  The backward keeps only two fp32 row vectors
+// there (D and the base-2 LSE), and its preprocess kernel rewrites both on
+// every call before anything reads them, so nothing carries over from one
+// call to the next; but two calls whose kernels overlap on the GPU (for
 // example on two streams) race on the array.
 namespace {
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
-void* g_noalloc_ptr[kMaxDevices] = {};
+std::atomic<void*> g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on the current device.  In host code
-// the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// Device address of the scratch array on the current device (a supported
+// device: the caller has checked it).  In host code the array's name is only
+// a host-side stand-in, so the address is looked up once per device (with
+// that device current) and published with a release store.
 fa_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-  if (g_noalloc_ptr[dev] == nullptr) {
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-      void* p = nullptr;
+    p = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
       e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
       if (e != cudaSuccess) return cuda_fail(e);
-      g_noalloc_ptr[dev] = p;
+      g_noalloc_ptr[dev].store(p, std::memory_order_release);
     }
   }
-  *out = g_noalloc_ptr[dev];
+  *out = p;
   return FA_OK;
 }
 
@@ -481,11 +490,18 @@ extern "C" fa_status fa_backward_noalloc(const void* q, const void* k, const voi
                                          const void* o, const void* dO, const float* lse,
                                          void* dq, void* dk, void* dv, int B, int H, int N,
                                          int d, float scale, int causal, void* stream) {
-  if (B < 1 || H < 1 || N < 1 || d < 1 || d > 128) return FA_ERR_INVALID_ARG;
+  // Shape first (the size formula assumes checked sizes), then the size
+  // limit (host arithmetic only), then the device: the array's address is
+  // only looked up on a device the library's kernels run on.
+  fa_status st = check_common(B, H, N, d, scale, FA_BF16);
+  if (st != FA_OK) return st;
   if (ws_layout(B, H, N, d).total > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES))
     return FA_ERR_WORKSPACE;  // the problem needs more scratch than the array holds
+  fa::Launch L;
+  st = device_context(stream, &L);
+  if (st != FA_OK) return st;
   void* scratch = nullptr;
-  fa_status st = noalloc_scratch(&scratch);
+  st = noalloc_scratch(&scratch);
   if (st != FA_OK) return st;
   return fa_backward_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, scratch,
                         static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES), FA_BF16, stream);

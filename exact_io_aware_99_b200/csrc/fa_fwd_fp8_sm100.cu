@@ -662,14 +662,22 @@ __global__ void __launch_bounds__(kQThreads) amax_kernel(const T* __restrict__ x
   if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(amax_bits, m);
 }
 
-// codes = RN_satfinite(x * (448 / amax)); the quotient and the product are
-// single fp32 operations rounded to nearest.
+// The factor that maps amax to 448: one fp32 quotient rounded to nearest.
+// When there is none (amax = 0, or amax so small that 448 / amax overflows
+// fp32, below about 1.3e-36) the tensor is taken as it is: factor 1,
+// descale 1.
+__device__ __forceinline__ float quant_factor(float amax) {
+  const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+  return isfinite(inv) ? inv : 1.f;
+}
+
+// codes = RN_satfinite(x * quant_factor(amax)); the product is one fp32
+// operation rounded to nearest.
 template <typename T>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(const T* __restrict__ x, size_t n,
                                                              const unsigned* amax_bits,
                                                              uint8_t* __restrict__ codes) {
-  const float amax = __uint_as_float(*amax_bits);
-  const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+  const float inv = quant_factor(__uint_as_float(*amax_bits));
   const size_t nv = n / 8;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   const size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -701,7 +709,9 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const T* __restrict
 
 __global__ void descale_kernel(float* descale) {
   const float amax = *descale;  // holds amax's bits until now
-  *descale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  // amax / 448 when the codes were scaled by 448 / amax, else 1
+  const bool scaled = amax > 0.f && isfinite(__fdiv_rn(448.f, amax));
+  *descale = scaled ? __fdiv_rn(amax, 448.f) : 1.f;
 }
 
 template <typename T>

@@ -272,7 +272,9 @@ FA_API fa_status fa_backward_noalloc(const void* q, const void* k, const void* v
  *   o           bf16 [B, H, N, d]; lse fp32 [B, H, N] (natural log).
  * Both products Q K^T and P V run as E4M3 x E4M3 with fp32 accumulation; the
  * softmax statistics are fp32 and the probabilities are rounded to E4M3
- * (relative error <= 2^-4 each) before P V.  The result approximates the
+ * before P V (error at most max(2^-4 p, 2^-10) for a probability p taken
+ * against the reference max: relative 2^-4 in E4M3's normal range, at most
+ * 2^-10 absolute among its subnormals, and values below 2^-10 flush to 0).  The result approximates the
  * exact attention of the dequantised inputs; the rounding of P bounds the
  * difference per element.  d in {64, 80, 128}; scale, causal, stream and
  * errors as fa_forward.
@@ -288,8 +290,10 @@ FA_API fa_status fa_forward_fp8(const void* q, const void* k, const void* v,
  * inputs (the pages fix no FP8 scaling; this is the plain per-tensor
  * reading): amax = max |x| over the n elements, codes[e] =
  * RN(x[e] * (448 / amax)) with saturation to +-448, *descale = amax / 448
- * (each quotient and product one fp32 operation rounded to nearest; amax = 0
- * gives codes 0 and descale 1).
+ * (each quotient and product one fp32 operation rounded to nearest).  When
+ * 448 / amax has no finite fp32 value (amax = 0, or amax below about
+ * 1.3e-36) the factor and *descale are 1: the codes are x rounded to E4M3 as
+ * it is (all such values round to signed zeros).
  *   x        device pointer, n elements of dtype FA_BF16 or FA_FP32,
  *            16-byte aligned.
  *   codes    device pointer, n bytes, 16-byte aligned.

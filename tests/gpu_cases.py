@@ -102,3 +102,23 @@ def check_backward(q, k, v, do, scale, causal, heads=None):
     for name, err in worst.items():
         assert err <= TOL_GRAD_REL, f"{name} max abs err / max|ref| = {err:.3g} > {TOL_GRAD_REL}"
     return worst
+
+
+def l2_group_heads(B, H, N, d, causal, kv_bytes=2):
+    """(b, h) pairs a work-order mistake of the persistent kernels would hit
+    first.  The kernels run heads in groups sized so that a group's K and V
+    (2 N d elements of kv_bytes each per head) fit a 64 MB (causal) or 32 MB
+    (non-causal) share of L2, group after group; a CTA takes further items
+    by cancelling CTAs that have not started, so the first head of each
+    group (where one group's items hand over to the next) and the whole last
+    group (the items taken over at the end of the launch) are the ones to
+    check.  Returned sorted, as (b, h) with bh = b H + h."""
+    BH = B * H
+    per_head = 2 * N * d * kv_bytes
+    share = (64 if causal else 32) << 20
+    g = max(1, min(BH, share // max(per_head, 1)))
+    picks = set(range(0, BH, g))
+    last = ((BH - 1) // g) * g
+    picks.update(range(last, BH))
+    return [divmod(bh, H) for bh in sorted(picks)]
+

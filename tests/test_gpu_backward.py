@@ -3,12 +3,11 @@ analytic backward on the same seeded inputs (the GPU's own forward supplies O
 and LSE, as in training)."""
 import math
 
-import numpy as np
 import pytest
 import torch
 
 import workloads
-from gpu_cases import check_backward
+from gpu_cases import check_backward, l2_group_heads
 
 pytestmark = pytest.mark.gpu
 
@@ -49,18 +48,12 @@ def test_bf16_backward_is_bitwise_reproducible():
         assert torch.equal(ga, gb)
 
 
-def _sample_heads(B, H, n, seed):
-    rs = np.random.default_rng(seed)
-    picks = {(0, 0), (B - 1, H - 1)}
-    while len(picks) < n:
-        picks.add((int(rs.integers(B)), int(rs.integers(H))))
-    return sorted(picks)
-
-
-@pytest.mark.parametrize("name,n_heads", [("causal_d128", 2), ("long_d128", 1),
-                                          ("gpt3_d80", 2)])
-def test_full_size_workload_backward(name, n_heads):
+# Full-size workloads in the benchmark's launch configuration: the first
+# head of every L2 head group and every head of the last group (see
+# gpu_cases.l2_group_heads) are checked completely.
+@pytest.mark.parametrize("name", ["causal_d128", "long_d128", "gpt3_d80"])
+def test_full_size_workload_backward(name):
     w = workloads.WORKLOADS[name]
     x = workloads.make_inputs(w)
     check_backward(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal,
-                   heads=_sample_heads(w.B, w.H, n_heads, w.seed + 1))
+                   heads=l2_group_heads(w.B, w.H, w.N, w.d, w.causal))

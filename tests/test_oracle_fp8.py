@@ -192,3 +192,21 @@ def test_quantize_generator_maps_amax_to_448():
     assert rel.max() <= 2.0 ** -4 + 1e-6
     c0, ds0 = workloads.quantize_e4m3(torch.zeros(5))
     assert ds0 == 1.0 and not c0.any()
+
+
+def test_quantize_generator_tiny_amax_takes_the_tensor_as_it_is():
+    # 448 / amax overflows fp32 for amax below ~1.3e-36: no factor maps amax
+    # to 448, so the factor and the descale are both 1 and every value
+    # (|x| < 2^-10) rounds to a signed zero -- never to a NaN code.
+    x = torch.tensor([0.0, 1e-37, -3e-37, 0.0, 5e-38, -0.0], dtype=torch.float32)
+    with np.errstate(over="ignore"):
+        assert not math.isfinite(np.float32(448.0) / np.float32(x.abs().max()))
+    c, ds = workloads.quantize_e4m3(x)
+    assert ds == 1.0
+    assert set(c.tolist()) <= {0x00, 0x80}
+    assert np.all(e4m3_decode(c.numpy()) == 0.0)
+    # just above the overflow point the ordinary rule applies
+    y = torch.tensor([0.0, 2e-36, -1e-36], dtype=torch.float32)
+    c1, ds1 = workloads.quantize_e4m3(y)
+    assert np.float32(ds1) == np.float32(2e-36) / np.float32(448.0)
+    assert np.abs(e4m3_decode(c1.numpy())).max() == 448.0

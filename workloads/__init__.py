@@ -197,13 +197,15 @@ def quantize_e4m3(x: torch.Tensor) -> Tuple[torch.Tensor, float]:
     """Per-tensor E4M3 quantisation of a float tensor (computed in fp32):
     amax = max |x|, descale = amax / 448 and codes = RN(x * (448 / amax)),
     each step one fp32 operation, the last through torch's float8_e4m3fn
-    conversion (round to nearest even); amax = 0 gives descale 1.  Returns
-    the codes as a contiguous uint8 tensor and the fp32 descale factor."""
+    conversion (round to nearest even).  When 448 / amax has no finite fp32
+    value (amax = 0, or amax below about 1.3e-36) the tensor is taken as it
+    is: factor 1, descale 1.  Returns the codes as a contiguous uint8 tensor
+    and the fp32 descale factor."""
     xf = x.float()
     amax = xf.abs().max() if xf.numel() else torch.tensor(0.0)
     lim = torch.tensor(E4M3_MAX, dtype=torch.float32)
-    if float(amax) > 0.0:
-        inv = lim / amax
+    inv = lim / amax if float(amax) > 0.0 else torch.tensor(float("inf"))
+    if bool(torch.isfinite(inv)):
         descale = float(amax / lim)
     else:
         inv = torch.tensor(1.0, dtype=torch.float32)
