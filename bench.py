@@ -5,9 +5,9 @@
                     [--impl ours|reference] [--no-cpu-baseline] [--sweep]
 
 One step is one pass of the whole hot path over one batch: the forward
-(fa_forward: O and LSE) followed by the backward (fa_backward: the D / LSE2
-preprocess, the dK/dV kernel and the dQ kernel) of the workload, inputs
-resident in HBM.  Throughput counts the algorithmic FLOPs of both passes
+(fa_forward: O and LSE) followed by the backward (fa_backward: the dQ
+kernel, which also forms the row statistics D and LSE2, then the dK/dV
+kernel) of the workload, inputs resident in HBM.  Throughput counts the algorithmic FLOPs of both passes
 (forward 4 B H N^2 d, halved when causal; backward 2.5x the forward).
 
 Default workload: causal_d128 (B4 H16 N4096 d128, bf16, causal fwd+bwd),
@@ -85,17 +85,56 @@ def whole_job_tflops(ws: int, flops_per_rank: float, ms: float) -> float:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+    """SM clock and throttle-reason samples taken while a timed region runs.
+
+    Read in-process through NVML (read-only queries) every ``period_s`` by a
+    background thread, so even a timed region of a few tens of milliseconds
+    gets a few dozen samples; falls back to ``nvidia-smi -lms 100`` when the
+    NVML bindings are missing.  Samples taken while the GPU reported itself
+    busy (NVML utilisation > 0) count as under load."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clocks-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown"}
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.001):
         self.gpu = gpu_index
+        self.period = period_s
         self.proc = None
         self.path = None
+        self.thread = None
+        self.rows = []
+        self.stop_evt = threading.Event()
+        self.nvml = None
+
+    def _sample_nvml(self, nv, h):
+        while not self.stop_evt.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                util = nv.nvmlDeviceGetUtilizationRates(h).gpu
+                self.rows.append((time.perf_counter(), float(sm), int(rs), int(util)))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.nvml = nv
+            self.thread = threading.Thread(target=self._sample_nvml, args=(nv, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -103,11 +142,30 @@ class ClockSampler:
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)  # let the sampler start
         except Exception:
             self.proc = None
 
     def stop(self):
         out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.nvml is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            rows = list(self.rows)
+            if not rows:
+                return out
+            load = [r for r in rows if r[3] > 0] or rows
+            reasons = set()
+            for r in load:
+                for bit, name in self.REASONS.items():
+                    if r[2] & bit:
+                        reasons.add(name)
+            out.update(sm_mhz=statistics.median(r[1] for r in load), sm_max_mhz=self.max_mhz,
+                       reasons=sorted(reasons), samples=len(rows),
+                       samples_under_load=len([r for r in rows if r[3] > 0]),
+                       sm_mhz_min=min(r[1] for r in load), source="nvml",
+                       period_ms=self.period * 1e3)
+            return out
         if self.proc is None:
             return out
         self.proc.terminate()
@@ -137,7 +195,7 @@ class ClockSampler:
                     reasons.add(n)
         out.update(sm_mhz=statistics.median(sm) if sm else None,
                    sm_max_mhz=max(mx) if mx else None, reasons=sorted(reasons),
-                   samples=len(rows))
+                   samples=len(rows), source="nvidia-smi")
         return out
 
 
@@ -240,7 +298,6 @@ def run_ours(args, peaks, peak_kind):
     barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
-    time.sleep(0.3)  # let the sampler start
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -309,6 +366,10 @@ def run_ours(args, peaks, peak_kind):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
+    extras = {}
+    if ws == 1 and not args.no_extras and args.workload == "causal_d128":
+        extras = run_extras(fa, dev, stream, peaks, local)
+
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -339,18 +400,185 @@ def run_ours(args, peaks, peak_kind):
         "frac_of_sustained_peak": round(value / ws / peak_s, 4),
         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json bf16_tflops burst {peak}, "
                        f"sustained {peak_s})",
-        "roofline": {"kernel": "fa_backward (preprocess + dK/dV kernel + dQ kernel)",
+        "roofline": {"kernel": "fa_backward (dQ kernel + dK/dV kernel)",
                      "bound": "tensor", "achieved": round(bwd_tf, 3), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(bwd_tf / peak, 4),
                      "traffic": traffic,
                      "algorithmic_bytes": perf.bwd_bytes(B, H, N, d)},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                    "reasons": clk["reasons"], "samples": clk["samples"]},
         "e2e": e2e,
         "cpu_baseline": cpu,
+        **extras,
     }
     return line
+
+
+# ------------------------------------------------------------------ extras
+# The other configurations, the TFLOP/s-vs-N curve and the FP8 and decode
+# paths, each timed in the same process with CUDA events on the launching
+# stream (3 warm-up steps, then every timed pass bracketed by its own events),
+# so one benchmark line carries all of them.  Forward-only working sets that
+# fit in L2 get a 256 MB write before every timed pass.
+
+EXTRA_ITERS = 10
+
+
+def _timed_passes(passes, stream, iters, flush=None):
+    """Mean device time (ms) of each callable in ``passes`` over ``iters``
+    rounds; every pass gets its own event pair (and an L2 flush first when
+    ``flush`` is given)."""
+    for _ in range(3):
+        for f in passes:
+            f()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in passes] for _ in range(iters)]
+    for i in range(iters):
+        for f, (a, b) in zip(passes, ev[i]):
+            if flush is not None:
+                flush.zero_()
+            a.record(stream)
+            f()
+            b.record(stream)
+    torch.cuda.synchronize()
+    return [statistics.mean(ev[i][p][0].elapsed_time(ev[i][p][1]) for i in range(iters))
+            for p in range(len(passes))]
+
+
+def _dense_entry(fa, dev, stream, B, H, N, d, causal, backward, inputs, peak, flush=None):
+    """Forward (and backward) TFLOP/s of one dense bf16 problem."""
+    q, k, v = (inputs[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    sp = stream.cuda_stream
+    sc = 1.0 / math.sqrt(d)
+
+    def f():
+        fa.fa_forward(q, k, v, o, lse, B, H, N, d, sc, causal, sp)
+    passes = [f]
+    if backward:
+        do = inputs["do"].to(dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        wb = fa.fa_backward_workspace_size(B, H, N, d)
+        wsb = torch.empty(wb, device=dev, dtype=torch.uint8)
+
+        def g():
+            fa.fa_backward(q, k, v, o, do, lse, dq, dk, dv, B, H, N, d, sc, causal, wsb, wb, sp)
+        passes.append(g)
+    ms = _timed_passes(passes, stream, EXTRA_ITERS, flush)
+    ff = perf.fwd_flops(B, H, N, d, causal)
+    out = {"B": B, "H": H, "N": N, "d": d, "causal": causal,
+           "fwd_ms": round(ms[0], 4), "fwd_tflops": round(ff / (ms[0] * 1e-3) / 1e12, 2)}
+    out["fwd_frac_of_peak"] = round(out["fwd_tflops"] / peak, 4)
+    if backward:
+        fb = perf.bwd_flops(B, H, N, d, causal)
+        out.update(bwd_ms=round(ms[1], 4), bwd_tflops=round(fb / (ms[1] * 1e-3) / 1e12, 2))
+        out["bwd_frac_of_peak"] = round(out["bwd_tflops"] / peak, 4)
+        out["step_tflops"] = round((ff + fb) / ((ms[0] + ms[1]) * 1e-3) / 1e12, 2)
+    if flush is not None:
+        out["l2"] = "flushed before every timed pass (256 MB write)"
+    return out
+
+
+def _device_randn(shape, seed, dev):
+    g = torch.Generator(device=dev).manual_seed(seed)
+    return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+
+def _projected_inputs(w, dev):
+    """The GPT-3-shaped workload's Q, K, V (X W projections) and dO, drawn
+    from the workload's seed on the CPU with the projections multiplied on
+    the GPU in fp32 (timing input only; the parity tests use the CPU
+    product)."""
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    x = torch.randn(w.B, w.N, w.hidden, generator=g, dtype=torch.float32).to(dev)
+    out = {}
+    for name in ("q", "k", "v"):
+        wm = (torch.randn(w.hidden, w.H * w.d, generator=g, dtype=torch.float32) * 0.02).to(dev)
+        pr = torch.matmul(x, wm).view(w.B, w.N, w.H, w.d).permute(0, 2, 1, 3).contiguous()
+        out[name] = pr.to(torch.bfloat16)
+    out["do"] = torch.randn(w.B, w.H, w.N, w.d, generator=g, dtype=torch.float32).to(
+        torch.bfloat16).to(dev)
+    return out
+
+
+def run_extras(fa, dev, stream, peaks, gpu_index):
+    peak = float(peaks["bf16_tflops"])
+    hbm = float(peaks.get("hbm_gbs", 6534.8))
+    flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
+    clocks = ClockSampler(gpu_index, period_s=0.005)
+    clocks.start()
+    configs = {}
+    w = workloads.WORKLOADS["fwd_d64"]
+    configs["fwd_d64"] = _dense_entry(fa, dev, stream, w.B, w.H, w.N, w.d, w.causal, False,
+                                      workloads.make_inputs(w), peak, flush)
+    for name in ("long_d128", "gpt3_d80"):
+        w = workloads.WORKLOADS[name]
+        x = _projected_inputs(w, dev) if w.projected else workloads.make_inputs(w)
+        configs[name] = _dense_entry(fa, dev, stream, w.B, w.H, w.N, w.d, w.causal, True, x,
+                                     peak)
+        del x
+    vs_n = []
+    for causal in (True, False):
+        for N in (512, 1024, 2048, 4096, 8192, 16384):
+            H, d = 16, 128
+            B = max(1, 262144 // (H * N))
+            x = {n: _device_randn((B, H, N, d), 5000 + 10 * N + i + 7 * causal, dev)
+                 for i, n in enumerate(("q", "k", "v", "do"))}
+            vs_n.append(_dense_entry(fa, dev, stream, B, H, N, d, causal, True, x, peak))
+            del x
+    # FP8 forward at the target shape (E4M3 codes from the library's own
+    # per-tensor quantiser), L2 flushed before every pass
+    w = workloads.WORKLOADS["fp8_causal_d128"]
+    q8, qd = fa.quantize_fp8(_device_randn((w.B, w.H, w.N, w.d), 7001, dev))
+    k8, kd = fa.quantize_fp8(_device_randn((w.B, w.H, w.N, w.d), 7002, dev))
+    v8, vd = fa.quantize_fp8(_device_randn((w.B, w.H, w.N, w.d), 7003, dev))
+    o8 = torch.empty((w.B, w.H, w.N, w.d), device=dev, dtype=torch.bfloat16)
+    l8 = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
+
+    def f8():
+        fa.fa_forward_fp8(q8, k8, v8, qd, kd, vd, o8, l8, w.B, w.H, w.N, w.d, w.scale, w.causal,
+                          stream.cuda_stream)
+    ms8 = _timed_passes([f8], stream, EXTRA_ITERS, flush)[0]
+    tf8 = perf.fwd_flops(w.B, w.H, w.N, w.d, w.causal) / (ms8 * 1e-3) / 1e12
+    fp8 = {"workload": w.describe(), "fwd_ms": round(ms8, 4), "fwd_tflops": round(tf8, 2),
+           "frac_of_fp8_peak": round(tf8 / (2 * peak), 4),
+           "fp8_peak": round(2 * peak, 1), "fp8_peak_source": "2 x measured bf16 (nominal ratio)",
+           "l2": "flushed before every timed pass (256 MB write)"}
+    del q8, k8, v8, o8
+    # split-KV decode (bound by reading K and V)
+    w = workloads.WORKLOADS["decode_d128"]
+    qd_ = _device_randn((w.B, w.H, w.N, w.d), 7101, dev)
+    kd_ = _device_randn((w.B, w.H, w.nk, w.d), 7102, dev)
+    vd_ = _device_randn((w.B, w.H, w.nk, w.d), 7103, dev)
+    od_ = torch.empty_like(qd_)
+    ld_ = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
+    splits = fa.fa_splitkv_default_splits(w.B, w.H, w.N, w.nk)
+    wb = fa.fa_splitkv_workspace_size(w.B, w.H, w.N, w.nk, w.d, splits)
+    wsb = torch.empty(wb, device=dev, dtype=torch.uint8)
+
+    def fdec():
+        fa.fa_forward_splitkv(qd_, kd_, vd_, od_, ld_, w.B, w.H, w.N, w.nk, w.d, w.scale,
+                              w.causal, splits, wsb, wb, stream.cuda_stream)
+    msd = _timed_passes([fdec], stream, EXTRA_ITERS)[0]
+    nbytes = perf.decode_bytes(w.B, w.H, w.N, w.nk, w.d)
+    gbs = nbytes / (msd * 1e-3) / 1e9
+    decode = {"workload": w.describe(), "num_splits": splits, "fwd_ms": round(msd, 4),
+              "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm, 4),
+              "tflops": round(perf.decode_flops(w.B, w.H, w.N, w.nk, w.d, w.causal)
+                              / (msd * 1e-3) / 1e12, 2),
+              "algorithmic_bytes": nbytes,
+              "l2": "K/V %.2f GB > 126 MB L2" % (2 * w.B * w.H * w.nk * w.d * 2 / 1e9)}
+    clk = clocks.stop()
+    st, site = fa.fa_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError(f"device wait timed out in the extra measurements (site {site:#x})")
+    return {"configs": configs, "vs_n": vs_n, "fp8_fwd": fp8, "decode": decode,
+            "extras_clocks": clk,
+            "extras_note": "each entry CUDA-event timed in this process after 3 warm-up "
+                           f"steps, mean of {EXTRA_ITERS} timed passes; fractions of the "
+                           "measured bf16 peak (burst)"}
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -393,7 +621,6 @@ def run_decode(args, peaks, peak_kind):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
-    time.sleep(0.3)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(args.steps):
@@ -529,7 +756,6 @@ def run_fp8(args, peaks, peak_kind):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
-    time.sleep(0.3)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     for a, b in evs:
@@ -774,6 +1000,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configs, the vs-N curve and the FP8/decode entries")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true", help="print the TFLOP/s-vs-N sweep instead")
     ap.add_argument("--splits", type=int, default=0,

@@ -93,14 +93,15 @@ fa_status get_encoder() {
   return g_encode ? FA_OK : FA_ERR_CUDA;
 }
 
-// [BH, N, d] bf16 viewed as 3-D {d, N, BH}; box {64, 128, 1}; 128-byte
-// swizzle; out-of-range rows and columns read as zero.
-fa_status make_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
+// [BH, N, d] bf16 viewed as 3-D {d, N, BH}; box {64, box_rows, 1}; 128-byte
+// swizzle; out-of-range rows and columns read as zero (loads) or are not
+// written (stores).
+fa_status make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows = 128) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -221,11 +222,12 @@ fa_status fa_forward_ex(const void* q, const void* k, const void* v, void* o, fl
   } else {
     st = get_encoder();
     if (st != FA_OK) return st;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
     if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
     if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
-    e = fa::launch_fwd_sm100(tq, tk, tv, o, lse, BH, N, d, scale, cz, nullptr, L);
+    if ((st = make_map(&to, o, BH, N, d, fa::kStoreBoxRows)) != FA_OK) return st;
+    e = fa::launch_fwd_sm100(tq, tk, tv, to, o, lse, BH, N, d, scale, cz, nullptr, L);
   }
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
@@ -250,12 +252,14 @@ fa_status fa_forward_blocksparse(const void* q, const void* k, const void* v, vo
   const int BH = B * H;
   st = get_encoder();
   if (st != FA_OK) return st;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
+  if ((st = make_map(&to, o, BH, N, d, fa::kStoreBoxRows)) != FA_OK) return st;
   const fa::BlockMaskArg bm{block_mask, mask_heads, H};
-  cudaError_t e = fa::launch_fwd_sm100(tq, tk, tv, o, lse, BH, N, d, scale, causal ? 1 : 0, &bm, L);
+  cudaError_t e =
+      fa::launch_fwd_sm100(tq, tk, tv, to, o, lse, BH, N, d, scale, causal ? 1 : 0, &bm, L);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
@@ -303,9 +307,8 @@ fa_status fa_backward_ex(const void* q, const void* k, const void* v, const void
   if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tdo, dO, BH, N, d)) != FA_OK) return st;
-  e = fa::launch_bwd_preprocess(o, dO, lse, dvec, lse2, BH, N, d, 1, L);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, d, scale, cz, nullptr, L);
+  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv, BH, N, d, scale,
+                           cz, nullptr, L);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
@@ -340,11 +343,9 @@ fa_status fa_backward_blocksparse(const void* q, const void* k, const void* v, c
   if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
   if ((st = make_map(&tdo, dO, BH, N, d)) != FA_OK) return st;
-  cudaError_t e = fa::launch_bwd_preprocess(o, dO, lse, dvec, lse2, BH, N, d, 1, L);
-  if (e != cudaSuccess) return cuda_fail(e);
   const fa::BlockMaskArg bm{block_mask, mask_heads, H};
-  e = fa::launch_bwd_sm100(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, d, scale,
-                           causal ? 1 : 0, &bm, L);
+  cudaError_t e = fa::launch_bwd_sm100(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv, BH, N,
+                                       d, scale, causal ? 1 : 0, &bm, L);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
@@ -450,8 +451,8 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
 // The array lives in device memory of every GPU that loads the library, for
 // the life of the process.  All calls on a GPU share it and it keeps the
 // previous call's contents.  The backward keeps only two fp32 row vectors
-// there (D and the base-2 LSE), and its preprocess kernel rewrites both on
-// every call before anything reads them, so nothing carries over from one
+// there (D and the base-2 LSE), and its dQ kernel rewrites both on every
+// call before the dK/dV kernel reads them, so nothing carries over from one
 // call to the next; but two calls whose kernels overlap on the GPU (for
 // example on two streams) race on the array.
 namespace {

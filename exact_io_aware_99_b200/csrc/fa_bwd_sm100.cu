@@ -19,23 +19,24 @@
 //  query tiles Q_i that see it.  Per Q tile:
 //      S^T  = K_j Q_i^T   (SS)  -> TMEM A = cols [0,128)
 //      dP^T = V_j dO_i^T  (SS)  -> TMEM B = cols [128,256)
-//      softmax warps: P^T = 2^(S^T c - LSE2) into already-read columns of A,
-//        dS^T = P^T o (dP^T - D) into already-read columns of B (bf16)
+//      softmax warps: P^T = 2^(S^T c - LSE2) and dS^T = P^T o (dP^T - D),
+//        both written (bf16) into B once dP^T has been read from it
 //      dV += P^T dO_i     (TS, P^T from TMEM)  -> cols [256,256+d)
 //      dK += dS^T Q_i     (TS, dS^T from TMEM) -> cols [384,384+d)
-//    issued as S_0, dP_0, [P_0] dV_0, S_1, [dS_0] dK_0, dP_1, [P_1] dV_1,
-//    S_2, [dS_1] dK_1, ... : S_{i+1} goes in right behind dV_i (which
-//    releases P_i's columns), so it is ready when the softmax finishes dS_i,
-//    and the softmax forms P_{i+1} while the tensor core runs dK_i, dP_{i+1}.
+//    A only ever holds S^T: as soon as the softmax has read S^T_i into
+//    registers, S^T_{i+1} is issued into A, so the tensor core computes it
+//    while the softmax still works on P^T_i.  Issue order S_0, dP_0,
+//    [S_0 read] S_1, [P_0] dV_0, [dS_0] dK_0, dP_1, [S_1 read] S_2, ...
 //  dQ kernel -- one CTA per (head, 128-query tile Q_i), looping over the key
 //  tiles K_j it sees.  Per key tile:
-//      S  = Q_i K_j^T     (SS)  -> TMEM S buffer j%2 (double-buffered)
-//      dP = dO_i V_j^T    (SS)  -> cols [256,384)
-//      softmax warps: dS = P o (dP - D), bf16, into read columns of S
+//      S  = Q_i K_j^T     (SS)  -> TMEM cols [0,128)
+//      dP = dO_i V_j^T    (SS)  -> dP buffer j%2, cols [128,256) or [256,384)
+//      softmax warps: dS = P o (dP - D), bf16, into the dP buffer it read
 //      dQ += dS K_j       (TS, dS from TMEM) -> cols [384,384+d)
-//  and dQ is written once, in bf16, at the end: no atomics and no fp32 dQ
-//  buffer, at the price of recomputing S and dP (7 tile MMAs per tile pair
-//  instead of 5).
+//    S_{j+1} is issued as soon as the softmax has read S_j, and dP_{j+1}
+//    right behind it into the other buffer.  dQ is written once, in bf16, at
+//    the end: no atomics and no fp32 dQ buffer, at the price of recomputing
+//    S and dP (7 tile MMAs per tile pair instead of 5).
 // Warp roles (both kernels, 10 warps): warps 0-3 and 4-7 are two softmax
 // warpgroups splitting the 128 columns of every tile in halves (one thread
 // per TMEM lane), warp 8 is the TMA producer, warp 9 the TMEM allocator and
@@ -53,15 +54,6 @@ namespace fa {
 namespace bwd {
 
 constexpr int kT = 128;  // rows of every tile (keys or queries)
-// Issue-order switches (both on; off gives the older, slower orders):
-// dK/dV kernel: S_{i+1} right after dV_i instead of after dS_i;
-// dQ kernel: dP_{j+1} ahead of dQ_j.
-#ifndef FA_BWD_EARLY_S
-#define FA_BWD_EARLY_S 1
-#endif
-#ifndef FA_BWD_EARLY_DP
-#define FA_BWD_EARLY_DP 1
-#endif
 // dK/dV kernel: one column pair in this many takes the FMA-pipe exp2 (0: none).
 #ifndef FA_BWD_POLY_EVERY
 #define FA_BWD_POLY_EVERY 0
@@ -234,25 +226,35 @@ __device__ __forceinline__ void dq_p_row(const uint32_t (&sv)[2][32], float scal
 template <int D>
 struct KvCfg : Shape<D> {
   using S = Shape<D>;
+  // S^T_{i+1} is issued as soon as the softmax has read S^T_i, about one
+  // iteration before dK_i releases Q_i's stage: Q needs three stages so that
+  // Q_{i+1} has landed by then.  dO_i is released by dV_i and first needed
+  // by dP_i at the end of iteration i - 1: two stages suffice.
+  static constexpr int NQ = 3, NDO = 2;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + S::TILE;
-  static constexpr int Q_OFF = V_OFF + S::TILE;       // [2] stages
-  static constexpr int DO_OFF = Q_OFF + 2 * S::TILE;  // [2] stages
-  // [2] stages of the query tile's LSE2 (512 B) then D (512 B)
-  static constexpr int VEC_OFF = DO_OFF + 2 * S::TILE;
-  static constexpr int BAR_OFF = VEC_OFF + 2 * 1024;
-  static constexpr int NBAR = 18;
+  static constexpr int Q_OFF = V_OFF + S::TILE;          // [NQ] stages
+  static constexpr int DO_OFF = Q_OFF + NQ * S::TILE;    // [NDO] stages
+  static constexpr int LSE_OFF = DO_OFF + NDO * S::TILE; // [NQ] x 512 B: the Q tile's LSE2
+  static constexpr int DV_OFF = LSE_OFF + NQ * 512;      // [NDO] x 512 B: the dO tile's D
+  static constexpr int BAR_OFF = DV_OFF + NDO * 512;
+  static constexpr int NBAR = 22;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
-  static constexpr int SMEM = MISC_OFF + 48 + 1024;
+  static constexpr int USED = MISC_OFF + 48;
+  // Slack for aligning the dynamic shared memory to 1 KB, as far as the
+  // budget allows; the kernel checks at run time that it was enough.
+  static constexpr int SLACK = USED + 1024 <= 232448 ? 1024 : 232448 - USED;
+  static constexpr int SMEM = USED + SLACK;
   static_assert(MISC_OFF % 16 == 0, "next-item responses need 16-byte alignment");
-  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(SLACK >= 0 && SMEM <= 232448, "shared memory budget");
 };
 
-// TMEM columns of the dK/dV kernel.  Region A holds S^T, region B dP^T;
-// softmax warpgroup h reads S^T columns [64h, 64h+64) and writes its P^T
-// (bf16 pairs) into [64h, 64h+32), then reads dP^T columns [128+64h, +64)
-// and writes its dS^T into [128+64h, 128+64h+32).
+// TMEM columns of the dK/dV kernel.  Region A holds S^T only, region B dP^T
+// and then the softmax results: warpgroup h reads S^T columns [64h, 64h+64)
+// of A and dP^T columns [128+64h, +64) of B, then writes its P^T (bf16
+// pairs) into [128+64h, +32) and its dS^T into [128+64h+32, +32).
 constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvColDV = 256, kKvColDK = 384;
+constexpr uint32_t kKvOffP = 0, kKvOffDS = 32;  // within a warpgroup's 64 columns of B
 
 template <int D, bool CAUSAL, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -266,23 +268,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                     WaitCtl ctl) {
   using C = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
+  {
+    // The budget may leave less than 1 KB of alignment slack (d = 80, 128):
+    // give up, recorded in the status word, if the base needs more.
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad > static_cast<uint32_t>(C::SLACK)) {
+      if (threadIdx.x == 0) atomicCAS(ctl.status, 0, kSiteBwdSmem);
+      return;
+    }
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;     // [2]
-  uint64_t* do_full = bars + 3;    // [2]
-  uint64_t* qdo_empty = bars + 5;  // [2]
-  uint64_t* s_full = bars + 7;
-  uint64_t* dp_full = bars + 8;
-  uint64_t* p_full = bars + 9;     // both softmax warpgroups wrote P^T
-  uint64_t* ds_full = bars + 10;   // both wrote dS^T (and are done with S^T, dP^T)
-  uint64_t* kv_done = bars + 11;   // the item's last dK: accumulators final
-  uint64_t* kv_empty = bars + 12;  // the item's S^T and dP^T MMAs are done with K_j, V_j
-  uint64_t* nxt_full = bars + 13;  // [2] next-item requests
-  uint64_t* nxt_empty = bars + 15; // [2]
+  uint64_t* q_full = bars + 1;     // [NQ]  Q_i and its LSE2
+  uint64_t* q_empty = bars + 4;    // [NQ]  dK_i is done with Q_i
+  uint64_t* do_full = bars + 7;    // [NDO] dO_i and its D
+  uint64_t* do_empty = bars + 9;   // [NDO] dV_i is done with dO_i
+  uint64_t* s_full = bars + 11;
+  uint64_t* dp_full = bars + 12;
+  uint64_t* p_full = bars + 13;    // both softmax warpgroups wrote P^T
+  uint64_t* ds_full = bars + 14;   // both wrote dS^T
+  uint64_t* kv_done = bars + 15;   // the item's last dK: accumulators final
+  uint64_t* kv_empty = bars + 16;  // the item's S^T and dP^T MMAs are done with K_j, V_j
+  uint64_t* nxt_full = bars + 17;  // [2] next-item requests
+  uint64_t* nxt_empty = bars + 19; // [2]
+  uint64_t* s_read = bars + 21;    // both softmax warpgroups have S^T in registers
   uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 36);
@@ -311,17 +324,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < C::NQ; ++s) {
       mbar_init(q_full + s, 1);
+      mbar_init(q_empty + s, 1);
+    }
+    for (int s = 0; s < C::NDO; ++s) {
       mbar_init(do_full + s, 1);
-      mbar_init(qdo_empty + s, 1);
+      mbar_init(do_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(nxt_full + s, 1);
       mbar_init(nxt_empty + s, 9);  // MMA warp + 8 softmax warps
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 2 * kT);
-    mbar_init(ds_full, 2 * kT);
+    // softmax-side barriers: one arrival per softmax warp
+    mbar_init(s_read, 8);
+    mbar_init(p_full, 8);
+    mbar_init(ds_full, 8);
     mbar_init(kv_done, 1);
     *abort = 0;
     fence_barrier_init();
@@ -349,7 +369,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
     }
-    int last[2] = {-1, -1};
+    int last_q[C::NQ], last_do[C::NDO];  // last ring use of each stage (drained on abort)
+#pragma unroll
+    for (int s = 0; s < C::NQ; ++s) last_q[s] = -1;
+#pragma unroll
+    for (int s = 0; s < C::NDO; ++s) last_do[s] = -1;
     int kv_issued = 0;
     int nxt_pending = -1;
     uint32_t nxt_pending_par = 0;
@@ -362,6 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         nxt_pending = -1;
         if (idx < 0) break;
       }
+      // Ask for item w + 1 right away, so its loads can follow this item's.
+      if (!producer_request_item(w, nxt_full, nxt_empty, nxt_resp, abort, ctl, kSiteBwdProducer,
+                                 leader, nxt_pending, nxt_pending_par))
+        break;
       int bh, j, i_start, n_iter;
       decode(idx, bh, j, i_start, n_iter);
       if (n_iter > 0) {
@@ -381,44 +409,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileCursor cur(n_t);
         for (int it = 0; it < n_iter; ++it, ++qr) {
           const int ic = BS ? cur.next(tiles) : i_start + it;  // query tile of the step
-          const int st = static_cast<int>(qr & 1);
-          const uint32_t u = qr >> 1;
-          if (qr >= 2 && !wait_all(qdo_empty + st, (u - 1) & 1, abort, ctl, kSiteBwdProducer)) {
+          const int y = ic * kT;
+          const size_t vrow = static_cast<size_t>(bh) * Np + y;
+          const int sq = static_cast<int>(qr % C::NQ), sd = static_cast<int>(qr % C::NDO);
+          const uint32_t uq = qr / C::NQ, ud = qr / C::NDO;
+          if (qr >= C::NQ && !wait_all(q_empty + sq, (uq - 1) & 1, abort, ctl, kSiteBwdProducer)) {
             ok = false;
             break;
           }
           if (leader) {
-            const int y = ic * kT;
-            mbar_arrive_expect_tx(q_full + st, C::TILE + 1024);
+            mbar_arrive_expect_tx(q_full + sq, C::TILE + 512);
 #pragma unroll
             for (int b = 0; b < C::NB; ++b)
-              tma_load_3d(&tm_q, q_full + st, smem + C::Q_OFF + st * C::TILE + b * C::BLK,
+              tma_load_3d(&tm_q, q_full + sq, smem + C::Q_OFF + sq * C::TILE + b * C::BLK,
                           b * 64, y, bh);
-            const size_t vrow = static_cast<size_t>(bh) * Np + y;
-            bulk_load_1d(smem + C::VEC_OFF + st * 1024, lse2 + vrow, 512, q_full + st);
-            bulk_load_1d(smem + C::VEC_OFF + st * 1024 + 512, dvec + vrow, 512, q_full + st);
-            mbar_arrive_expect_tx(do_full + st, C::TILE);
-#pragma unroll
-            for (int b = 0; b < C::NB; ++b)
-              tma_load_3d(&tm_do, do_full + st, smem + C::DO_OFF + st * C::TILE + b * C::BLK,
-                          b * 64, y, bh);
+            bulk_load_1d(smem + C::LSE_OFF + sq * 512, lse2 + vrow, 512, q_full + sq);
           }
           __syncwarp();
-          last[st] = static_cast<int>(u);
+          last_q[sq] = static_cast<int>(uq);
+          if (qr >= C::NDO &&
+              !wait_all(do_empty + sd, (ud - 1) & 1, abort, ctl, kSiteBwdProducer)) {
+            ok = false;
+            break;
+          }
+          if (leader) {
+            mbar_arrive_expect_tx(do_full + sd, C::TILE + 512);
+#pragma unroll
+            for (int b = 0; b < C::NB; ++b)
+              tma_load_3d(&tm_do, do_full + sd, smem + C::DO_OFF + sd * C::TILE + b * C::BLK,
+                          b * 64, y, bh);
+            bulk_load_1d(smem + C::DV_OFF + sd * 512, dvec + vrow, 512, do_full + sd);
+          }
+          __syncwarp();
+          last_do[sd] = static_cast<int>(ud);
         }
         if (!ok) break;
       }
-      if (!producer_request_item(w, nxt_full, nxt_empty, nxt_resp, abort, ctl, kSiteBwdProducer,
-                                 leader, nxt_pending, nxt_pending_par))
-        break;
     }
     if (*abort && leader) {
       if (kv_issued > 0) drain_wait(kv_full, static_cast<uint32_t>(kv_issued - 1) & 1, ctl);
-      for (int s = 0; s < 2; ++s)
-        if (last[s] >= 0) {
-          drain_wait(q_full + s, last[s] & 1, ctl);
-          drain_wait(do_full + s, last[s] & 1, ctl);
-        }
+      for (int s = 0; s < C::NQ; ++s)
+        if (last_q[s] >= 0) drain_wait(q_full + s, last_q[s] & 1, ctl);
+      for (int s = 0; s < C::NDO; ++s)
+        if (last_do[s] >= 0) drain_wait(do_full + s, last_do[s] & 1, ctl);
       if (nxt_pending >= 0) drain_wait(nxt_full + nxt_pending, nxt_pending_par, ctl);
     }
     __syncwarp();
@@ -445,11 +478,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto issue_s = [&](int it) -> bool {  // S^T = K_j Q_i^T -> region A
       const uint32_t g = qbase + it;
-      const int st = static_cast<int>(g & 1);
-      if (!wait_all(q_full + st, (g >> 1) & 1, abort, ctl, kSiteBwdMma)) return false;
+      const int sq = static_cast<int>(g % C::NQ);
+      if (!wait_all(q_full + sq, (g / C::NQ) & 1, abort, ctl, kSiteBwdMma)) return false;
       tc_fence_after();
       if (leader) {
-        const SDesc qd = q_desc + st * C::TILE;
+        const SDesc qd = q_desc + sq * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
@@ -464,11 +497,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto issue_dp = [&](int it) -> bool {  // dP^T = V_j dO_i^T -> region B
       const uint32_t g = qbase + it;
-      const int st = static_cast<int>(g & 1);
-      if (!wait_all(do_full + st, (g >> 1) & 1, abort, ctl, kSiteBwdMma)) return false;
+      const int sd = static_cast<int>(g % C::NDO);
+      if (!wait_all(do_full + sd, (g / C::NDO) & 1, abort, ctl, kSiteBwdMma)) return false;
       tc_fence_after();
       if (leader) {
-        const SDesc dd = do_desc + st * C::TILE;
+        const SDesc dd = do_desc + sd * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
@@ -481,9 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       release_kv();
       return true;
     };
-    // S^T_{i+1} overwrites P^T_i in A: issued after dV_i (same thread, in
-    // order); the softmax is done with A once it signalled p_full.
-    // dP^T_{i+1} overwrites dS^T_i in B: issued after dK_i, in order.
+    // S^T_{i+1} overwrites S^T_i in A once both warpgroups have read it
+    // (s_read).  dP^T_{i+1} overwrites P^T_i and dS^T_i in B: issued after
+    // dV_i and dK_i (same thread, in order), which read them.
     bool ok = true;
     int idx = 0;
     uint32_t kv_items = 0;  // items with at least one query tile (one K/V load each)
@@ -499,11 +532,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++kv_items;
       for (int it = 0; ok && it < n_iter; ++it) {
         const uint32_t g = qbase + it;
-        const int st = static_cast<int>(g & 1);
-        const SDesc qm = q_mn + st * C::TILE;
-        const SDesc dm = do_mn + st * C::TILE;
+        const int sq = static_cast<int>(g % C::NQ), sd = static_cast<int>(g % C::NDO);
+        const SDesc qm = q_mn + sq * C::TILE;
+        const SDesc dm = do_mn + sd * C::TILE;
+        if (it + 1 < n_iter) {
+          if (!wait_all(s_read, g & 1, abort, ctl, kSiteBwdMma) || !issue_s(it + 1)) {
+            ok = false;
+            break;
+          }
+        }
         // dV += P^T dO_i: query k-step kk (16 queries) lives in columns
-        // 64*(kk/4) + 8*(kk%4) of region A.
+        // 64*(kk/4) + 8*(kk%4) of the P^T half of B.
         if (!wait_all(p_full, g & 1, abort, ctl, kSiteBwdMma)) {
           ok = false;
           break;
@@ -512,32 +551,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < kT / 16; ++kk)
-            mma_ts(tmem + kKvColDV, tmem + kKvColS + (kk >> 2) * 64 + (kk & 3) * 8,
+            mma_ts(tmem + kKvColDV, tmem + kKvColDP + kKvOffP + (kk >> 2) * 64 + (kk & 3) * 8,
                    dm + kk * 2048, kIdescAcc,
                    (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(do_empty + sd);
         }
         __syncwarp();
-        if (FA_BWD_EARLY_S && it + 1 < n_iter && !issue_s(it + 1)) {
-          ok = false;
-          break;
-        }
         if (!wait_all(ds_full, g & 1, abort, ctl, kSiteBwdMma)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (!FA_BWD_EARLY_S && it + 1 < n_iter && !issue_s(it + 1)) {
-          ok = false;
-          break;
-        }
-        // dK += dS^T Q_i: dS^T k-step kk at column 128 + 64*(kk/4) + 8*(kk%4).
+        // dK += dS^T Q_i: dS^T k-step kk at column 64*(kk/4) + 8*(kk%4) of
+        // the dS^T half of B.
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < kT / 16; ++kk)
-            mma_ts(tmem + kKvColDK, tmem + kKvColDP + (kk >> 2) * 64 + (kk & 3) * 8,
+            mma_ts(tmem + kKvColDK, tmem + kKvColDP + kKvOffDS + (kk >> 2) * 64 + (kk & 3) * 8,
                    qm + kk * 2048, kIdescAcc,
                    (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(qdo_empty + st);
+          mma_commit(q_empty + sq);
         }
         __syncwarp();
         if (it + 1 < n_iter && !issue_dp(it + 1)) {
@@ -556,12 +589,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2;
     const int kr = threadIdx.x & 127;  // key row == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t col_s = kKvColS + 64 * h;    // this half's S^T, then P^T
-    const uint32_t col_dp = kKvColDP + 64 * h;  // this half's dP^T, then dS^T
+    const uint32_t col_s = kKvColS + 64 * h;    // this half's S^T
+    const uint32_t col_dp = kKvColDP + 64 * h;  // this half's dP^T, then P^T and dS^T
     uint32_t qbase = 0;     // query tiles of the previous items (barrier phases)
     uint32_t kv_items = 0;  // items with at least one query tile
     bool ok = true;
     int idx = 0;
+    // One arrival per warp once every lane's tcgen05 loads / stores are done.
+    auto warp_arrive = [&](uint64_t* bar) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
     for (int w = 0; ok; ++w) {
       if (!next_item(w, idx, kSiteBwdSoftmax)) break;
       if (idx < 0) break;
@@ -583,11 +622,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < n_iter; ++it) {
         const int i = BS ? cur.next(tiles) : i_start + it;  // query tile of the step
         const uint32_t g = qbase + it;
-        const int st = static_cast<int>(g & 1);
         // LSE2 and D of this half's 64 queries, staged by the producer with
-        // the Q tile (q_full[st] completed before S^T, hence before s_full).
-        const float* l2 = reinterpret_cast<const float*>(smem + C::VEC_OFF + st * 1024) + 64 * h;
-        const float* dd = l2 + 128;
+        // the Q tile (q_full completed before S^T, hence before s_full) and
+        // the dO tile (do_full completed before dP^T, hence before dp_full).
+        const float* l2 =
+            reinterpret_cast<const float*>(smem + C::LSE_OFF + (g % C::NQ) * 512) + 64 * h;
+        const float* dd =
+            reinterpret_cast<const float*>(smem + C::DV_OFF + (g % C::NDO) * 512) + 64 * h;
         const bool diag = CAUSAL && (i == j);
         if (!wait_all(s_full, g & 1, abort, ctl, kSiteBwdSoftmax)) {
           ok = false;
@@ -598,6 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + col_s, sv[0]);
         tmem_ld32(lane_base + col_s + 32, sv[1]);
         tmem_wait_ld();
+        warp_arrive(s_read);  // A may take S^T_{i+1} now
         const float2 sc2 = make_float2(scale_log2, scale_log2);
         // queries of this half this key row sees: all, none (key past N), or
         // q >= key on the diagonal tile
@@ -607,11 +649,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           kv_p_row<true>(sv, l2, sc2, qlo, pk);
         else
           kv_p_row<false>(sv, l2, sc2, qlo, pk);
-        // P^T -> columns [col_s, col_s + 32): already read above.
-        tmem_st32(lane_base + col_s, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full);
 
         if (!wait_all(dp_full, g & 1, abort, ctl, kSiteBwdSoftmax)) {
           ok = false;
@@ -622,6 +659,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + col_dp, dpv[0]);
         tmem_ld32(lane_base + col_dp + 32, dpv[1]);
         tmem_wait_ld();
+        // P^T -> the first 32 of this half's dP^T columns (just read).
+        tmem_st32(lane_base + col_dp + kKvOffP, pk);
+        tmem_wait_st();
+        warp_arrive(p_full);
         uint32_t dsk[32];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -637,11 +678,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             dsk[c * 16 + e / 2 + 1] = pack_bf16(d2, d3);
           }
         }
-        // dS^T -> columns [col_dp, col_dp + 32): dP^T values there were read.
-        tmem_st32(lane_base + col_dp, dsk);
+        // dS^T -> the last 32 of this half's dP^T columns.
+        tmem_st32(lane_base + col_dp + kKvOffDS, dsk);
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(ds_full);
+        warp_arrive(ds_full);
       }
       if (!ok) break;
       // Epilogue: dV (unscaled) and dK (times scale), 16-column steps split
@@ -683,17 +723,18 @@ struct QCfg : Shape<D> {
   static constexpr int K_OFF = DO_OFF + S::TILE;      // [NK]
   static constexpr int V_OFF = K_OFF + NK * S::TILE;  // [NV]
   static constexpr int BAR_OFF = V_OFF + NV * S::TILE;
-  static constexpr int NBAR = 12 + 2 * NK + 2 * NV;
+  static constexpr int NBAR = (13 + 2 * NK + 2 * NV + 1) & ~1;  // even: keeps MISC 16-byte aligned
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
   static constexpr int SMEM = MISC_OFF + 48 + 1024;
   static_assert(MISC_OFF % 16 == 0, "next-item responses need 16-byte alignment");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-// TMEM columns of the dQ kernel: S double buffer, dP, dQ accumulator.
-// Softmax warpgroup h reads S columns [64h, 64h+64) of the current buffer and
-// writes its dS (bf16 pairs) into [64h, 64h+32) of the same buffer.
-constexpr uint32_t kQColS = 0, kQColDP = 256, kQColDQ = 384;
+// TMEM columns of the dQ kernel: S, two dP buffers, dQ accumulator.
+// Softmax warpgroup h reads S columns [64h, 64h+64) and dP columns
+// [64h, 64h+64) of the current dP buffer, and writes its dS (bf16 pairs) into
+// [64h, 64h+32) of that dP buffer.
+constexpr uint32_t kQColS = 0, kQColDP = 128, kQColDQ = 384;
 
 template <int D, bool CAUSAL, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -717,10 +758,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = k_full + C::NK;   // [NK]
   uint64_t* v_full = k_empty + C::NK;   // [NV]
   uint64_t* v_empty = v_full + C::NV;   // [NV]
-  uint64_t* s_full = v_empty + C::NV;   // [2] per S buffer
-  uint64_t* ds_full = s_full + 2;       // [2] per S buffer
-  uint64_t* dp_full = ds_full + 2;
-  uint64_t* nxt_full = dp_full + 1;     // [2] next-item requests
+  uint64_t* s_full = v_empty + C::NV;
+  uint64_t* s_read = s_full + 1;        // both softmax warpgroups have S in registers
+  uint64_t* dp_full = s_read + 1;       // [2] per dP buffer
+  uint64_t* ds_full = dp_full + 2;      // [2] per dP buffer
+  uint64_t* nxt_full = ds_full + 2;     // [2] next-item requests
   uint64_t* nxt_empty = nxt_full + 2;   // [2]
   uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
@@ -761,12 +803,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(v_empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full + b, 1);
-      mbar_init(ds_full + b, 2 * kT);
+      mbar_init(dp_full + b, 1);
+      mbar_init(ds_full + b, 8);    // one arrival per softmax warp
       mbar_init(nxt_full + b, 1);
       mbar_init(nxt_empty + b, 9);  // MMA warp + 8 softmax warps
     }
-    mbar_init(dp_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 8);
     *abort = 0;
     fence_barrier_init();
   }
@@ -810,6 +853,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         nxt_pending = -1;
         if (idx < 0) break;
       }
+      // Ask for item it + 1 right away, so its loads can follow this item's.
+      if (!producer_request_item(it, nxt_full, nxt_empty, nxt_resp, abort, ctl, kSiteBwdProducer,
+                                 leader, nxt_pending, nxt_pending_par))
+        break;
       int bh, i, n_kv;
       decode(idx, bh, i, n_kv);
       if (n_kv > 0) {
@@ -860,9 +907,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
       }
-      if (!producer_request_item(it, nxt_full, nxt_empty, nxt_resp, abort, ctl, kSiteBwdProducer,
-                                 leader, nxt_pending, nxt_pending_par))
-        break;
     }
     if (*abort && leader) {
       if (q_issued > 0) drain_wait(q_full, static_cast<uint32_t>(q_issued - 1) & 1, ctl);
@@ -885,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const SDesc v_desc = sdesc(sbase + C::V_OFF, 16, 1024);     // K-major (B of dP)
     const SDesc k_mn = sdesc(sbase + C::K_OFF, C::BLK, 1024);   // MN-major (B of dQ)
     // Running counts across items: key tiles (ring uses) before this item,
-    // which also number the S buffers (buffer g & 1 for the g-th S).
+    // which also number the dP buffers (buffer g & 1 for the g-th dP).
     uint32_t kbase = 0;
     int n_kv = 0, released = 0, s_done = 0, dp_done = 0;
     auto release_q = [&]() {  // after the item's last S and dP
@@ -895,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         released = 1;
       }
     };
-    auto issue_s = [&](int jj) -> bool {  // S_jj = Q K_jj^T -> buffer g % 2
+    auto issue_s = [&](int jj) -> bool {  // S_jj = Q K_jj^T -> S columns
       const uint32_t g = kbase + jj;
       const int s = static_cast<int>(g % C::NK);
       if (!wait_all(k_full + s, (g / C::NK) & 1, abort, ctl, kSiteBwdMma)) return false;
@@ -905,17 +949,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kQColS + (g & 1) * kT, q_desc + off, kd + off, kIdescSq,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kQColS, q_desc + off, kd + off, kIdescSq, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full + (g & 1));
+        mma_commit(s_full);
       }
       __syncwarp();
       ++s_done;
       release_q();
       return true;
     };
-    auto issue_dp = [&](int jj) -> bool {  // dP_jj = dO V_jj^T, then V_jj is free
+    auto issue_dp = [&](int jj) -> bool {  // dP_jj = dO V_jj^T -> buffer g % 2, then V_jj is free
       const uint32_t g = kbase + jj;
       const int s = static_cast<int>(g % C::NV);
       if (!wait_all(v_full + s, (g / C::NV) & 1, abort, ctl, kSiteBwdMma)) return false;
@@ -925,9 +968,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(tmem + kQColDP, do_desc + off, vd + off, kIdescSq, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kQColDP + (g & 1) * kT, do_desc + off, vd + off, kIdescSq,
+                 kk > 0 ? 1u : 0u);
         }
-        mma_commit(dp_full);
+        mma_commit(dp_full + (g & 1));
         mma_commit(v_empty + s);
       }
       __syncwarp();
@@ -935,12 +979,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       release_q();
       return true;
     };
-    // Order: S_0, dP_0, S_1, [dS_0] dP_1, dQ_0, S_2, [dS_1] dP_2, dQ_1, ...
-    // so the tensor core computes S_{j+1} while the softmax warps form dS_j,
-    // and dP_{j+1} is ready soon after.  S_{j+2} reuses S_j's buffer after
-    // dQ_j has read dS_j (same thread, in order) and the softmax released it
-    // (ds_full waited); dP_{j+1} overwrites dP_j once ds_full(j) says the
-    // softmax has read it.
+    // Order: S_0, dP_0, [S_0 read] S_1, dP_1, [dS_0] dQ_0, [S_1 read] S_2,
+    // dP_2, [dS_1] dQ_1, ...: S_{j+1} overwrites S_j once both warpgroups
+    // have read it, so the tensor core computes it while the softmax forms
+    // dS_j; dP_{j+1} overwrites dS_{j-1} in the other buffer after dQ_{j-1}
+    // has read it (same thread, in order).
     bool ok = true;
     int idx = 0;
     uint32_t q_items = 0;  // items with at least one key tile (one Q load each)
@@ -953,39 +996,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       released = s_done = dp_done = 0;
       ok = wait_all(q_full, q_items & 1, abort, ctl, kSiteBwdMma) && issue_s(0) && issue_dp(0);
       ++q_items;
-      if (ok && n_kv > 1) ok = issue_s(1);
       for (int jj = 0; ok && jj < n_kv; ++jj) {
         const uint32_t g = kbase + jj;
         const int s = static_cast<int>(g % C::NK);
+        if (jj + 1 < n_kv) {
+          if (!wait_all(s_read, g & 1, abort, ctl, kSiteBwdMma) || !issue_s(jj + 1) ||
+              !issue_dp(jj + 1)) {
+            ok = false;
+            break;
+          }
+        }
         if (!wait_all(ds_full + (g & 1), (g >> 1) & 1, abort, ctl, kSiteBwdMma)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (FA_BWD_EARLY_DP && jj + 1 < n_kv && !issue_dp(jj + 1)) {
-          ok = false;
-          break;
-        }
         // dQ += dS_jj K_jj: key k-step kk (16 keys) of dS at column
-        // 64*(kk/4) + 8*(kk%4) of the S buffer.
+        // 64*(kk/4) + 8*(kk%4) of the dP buffer.
         if (leader) {
           const SDesc km = k_mn + s * C::TILE;
 #pragma unroll
           for (int kk = 0; kk < kT / 16; ++kk)
-            mma_ts(tmem + kQColDQ, tmem + kQColS + (g & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
+            mma_ts(tmem + kQColDQ, tmem + kQColDP + (g & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
                    km + kk * 2048, kIdescDq,
                    (jj > 0 || kk > 0) ? 1u : 0u);
           mma_commit(k_empty + s);
         }
         __syncwarp();
-        if (!FA_BWD_EARLY_DP && jj + 1 < n_kv && !issue_dp(jj + 1)) {
-          ok = false;
-          break;
-        }
-        if (jj + 2 < n_kv && !issue_s(jj + 2)) {
-          ok = false;
-          break;
-        }
       }
       if (!ok) break;
       if (leader) mma_commit(dq_done);
@@ -998,7 +1035,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2;
     const int qr = threadIdx.x & 127;  // query row == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    uint32_t kbase = 0;    // key tiles of the previous items (S buffer numbering)
+    // One arrival per warp once every lane's tcgen05 loads / stores are done.
+    auto warp_arrive = [&](uint64_t* bar) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+    uint32_t kbase = 0;    // key tiles of the previous items (dP buffer numbering)
     uint32_t q_items = 0;  // items with at least one key tile
     bool ok = true;
     int idx = 0;
@@ -1022,16 +1065,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int jj = 0; jj < n_kv; ++jj) {
         const int jt = BS ? cur.next(tiles) : jj;  // key tile of the step
         const uint32_t g = kbase + jj;
-        const uint32_t col_s = kQColS + (g & 1) * kT + 64 * h;
-        if (!wait_all(s_full + (g & 1), (g >> 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
+        const uint32_t col_dp = kQColDP + (g & 1) * kT + 64 * h;
+        if (!wait_all(s_full, g & 1, abort, ctl, kSiteBwdSoftmax)) {
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t sv[2][32];
-        tmem_ld32(lane_base + col_s, sv[0]);
-        tmem_ld32(lane_base + col_s + 32, sv[1]);
+        tmem_ld32(lane_base + kQColS + 64 * h, sv[0]);
+        tmem_ld32(lane_base + kQColS + 64 * h + 32, sv[1]);
         tmem_wait_ld();
+        warp_arrive(s_read);  // the S columns may take S_{j+1} now
         const int k0 = jt * kT + 64 * h;  // first key of this half
         // keys k visible to this query: k <= q_idx (causal) and k < N
         const int lim = min(N, CAUSAL ? q_idx + 1 : N) - k0;
@@ -1040,14 +1084,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           dq_p_row<true>(sv, scale_log2, my_l2, lim, p);
         else
           dq_p_row<false>(sv, scale_log2, my_l2, lim, p);
-        if (!wait_all(dp_full, g & 1, abort, ctl, kSiteBwdSoftmax)) {
+        if (!wait_all(dp_full + (g & 1), (g >> 1) & 1, abort, ctl, kSiteBwdSoftmax)) {
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t dpv[2][32];
-        tmem_ld32(lane_base + kQColDP + 64 * h, dpv[0]);
-        tmem_ld32(lane_base + kQColDP + 64 * h + 32, dpv[1]);
+        tmem_ld32(lane_base + col_dp, dpv[0]);
+        tmem_ld32(lane_base + col_dp + 32, dpv[1]);
         tmem_wait_ld();
         uint32_t dsk[32];
 #pragma unroll
@@ -1057,11 +1101,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float d1 = p[c1] * (__uint_as_float(dpv[c1 >> 5][c1 & 31]) - my_d);
           dsk[c] = pack_bf16(d0, d1);
         }
-        // dS -> columns [col_s, col_s + 32) of the S buffer (already read).
-        tmem_st32(lane_base + col_s, dsk);
+        // dS -> the first 32 of this half's dP columns (already read).
+        tmem_st32(lane_base + col_dp, dsk);
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(ds_full + (g & 1));
+        warp_arrive(ds_full + (g & 1));
       }
       if (!ok) break;
       // dq_done completes once per item; the next item's first dQ MMA
@@ -1097,11 +1140,61 @@ inline int heads_per_group(long long per_head_bytes, int BH, bool causal) {
   return g < 1 ? 1 : (g > BH ? BH : g);
 }
 
+// Row statistics of the backward, one pass over O and dO: D = rowsum(dO o O)
+// (fp32, columns in order) and LSE2 = LSE log2(e), in [BH, Np] vectors
+// (Np = N rounded up to 128; rows past N get D = 0 and LSE2 = +inf, so a
+// whole 128-row tile can be read without masks).  Half a warp per row, each
+// lane one 16-byte piece of O and of dO (d / 8 lanes in use), so every load
+// instruction moves whole rows.
+template <int D>
+__global__ void __launch_bounds__(256) row_stats_kernel(const __nv_bfloat16* __restrict__ o,
+                                                        const __nv_bfloat16* __restrict__ dO,
+                                                        const float* __restrict__ lse,
+                                                        float* __restrict__ dvec,
+                                                        float* __restrict__ lse2, int BH, int N,
+                                                        int Np) {
+  constexpr int kPieces = D / 8;  // 16-byte pieces per row
+  static_assert(kPieces <= 16, "a row must fit half a warp");
+  const int lane = threadIdx.x & 31, sub = lane & 15;
+  const long long rows = static_cast<long long>(BH) * Np;
+  const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  // Warp w handles rows 2w and 2w + 1 (one per half); all lanes take the
+  // same trips, so the shuffles below always see the whole warp.
+  for (long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       2 * w < rows; w += nwarps) {
+    const long long r = 2 * w + (lane >> 4);
+    const bool in = r < rows;
+    const int bh = in ? static_cast<int>(r / Np) : 0;
+    const int row = in ? static_cast<int>(r - static_cast<long long>(bh) * Np) : N;
+    float acc = 0.f;
+    if (row < N && sub < kPieces) {
+      const size_t off = (static_cast<size_t>(bh) * N + row) * D + 8 * sub;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + off));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dO + off));
+      acc = fmaf(bf16lo(a.x), bf16lo(b.x), acc);
+      acc = fmaf(bf16hi(a.x), bf16hi(b.x), acc);
+      acc = fmaf(bf16lo(a.y), bf16lo(b.y), acc);
+      acc = fmaf(bf16hi(a.y), bf16hi(b.y), acc);
+      acc = fmaf(bf16lo(a.z), bf16lo(b.z), acc);
+      acc = fmaf(bf16hi(a.z), bf16hi(b.z), acc);
+      acc = fmaf(bf16lo(a.w), bf16lo(b.w), acc);
+      acc = fmaf(bf16hi(a.w), bf16hi(b.w), acc);
+    }
+#pragma unroll
+    for (int m = 8; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (in && sub == 0) {
+      dvec[r] = row < N ? acc : 0.f;
+      lse2[r] = row < N ? lse[static_cast<size_t>(bh) * N + row] * 1.4426950408889634f
+                        : INFINITY;
+    }
+  }
+}
+
 template <int D, bool CAUSAL, bool BS>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const CUtensorMap& tdo, const float* dvec, const float* lse2, void* dq,
-                   void* dk, void* dv, int BH, int N, float scale, const BlockMaskArg& bm,
-                   const Launch& L) {
+                   const CUtensorMap& tdo, const void* o, const void* dO, const float* lse,
+                   float* dvec, float* lse2, void* dq, void* dk, void* dv, int BH, int N,
+                   float scale, const BlockMaskArg& bm, const Launch& L) {
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, CAUSAL, BS>,
@@ -1119,53 +1212,66 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   const int group = heads_per_group(4LL * N * D, BH, CAUSAL);
   const float scale_log2 = scale * 1.4426950408889634f;
   WaitCtl ctl{L.status, L.limit_ns};
-  bwd_dkdv_kernel<D, CAUSAL, BS>
-      <<<static_cast<unsigned>(blocks), kThreads, KvCfg<D>::SMEM, L.stream>>>(
-          tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dk),
-          static_cast<__nv_bfloat16*>(dv), N, BH, group, scale, scale_log2, bm.mask,
-          bm.mask_heads, bm.H, ctl);
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long rows = static_cast<long long>(BH) * n_t * kT;
+  const long long want = (rows + 15) / 16;  // 16 rows per 256-thread block
+  const unsigned sblocks =
+      static_cast<unsigned>(want < 8LL * sms ? (want < 1 ? 1 : want) : 8LL * sms);
+  row_stats_kernel<D><<<sblocks, 256, 0, L.stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
+      lse2, BH, N, n_t * kT);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bwd_dq_kernel<D, CAUSAL, BS>
       <<<static_cast<unsigned>(blocks), kThreads, QCfg<D>::SMEM, L.stream>>>(
           tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dq), N, BH, group, scale,
           scale_log2, bm.mask, bm.mask_heads, bm.H, ctl);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dkdv_kernel<D, CAUSAL, BS>
+      <<<static_cast<unsigned>(blocks), kThreads, KvCfg<D>::SMEM, L.stream>>>(
+          tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dk),
+          static_cast<__nv_bfloat16*>(dv), N, BH, group, scale, scale_log2, bm.mask,
+          bm.mask_heads, bm.H, ctl);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                     const CUtensorMap& tdo, const float* dvec, const float* lse2, void* dq,
-                     void* dk, void* dv, int BH, int N, float scale, int causal,
-                     const BlockMaskArg* bm, const Launch& L) {
+                     const CUtensorMap& tdo, const void* o, const void* dO, const float* lse,
+                     float* dvec, float* lse2, void* dq, void* dk, void* dv, int BH, int N,
+                     float scale, int causal, const BlockMaskArg* bm, const Launch& L) {
   const BlockMaskArg none{nullptr, 1, 1};
   if (bm && bm->mask)
-    return causal ? launch<D, true, true>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale,
-                                          *bm, L)
-                  : launch<D, false, true>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale,
-                                           *bm, L);
-  return causal ? launch<D, true, false>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale,
-                                         none, L)
-                : launch<D, false, false>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale,
-                                          none, L);
+    return causal ? launch<D, true, true>(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv,
+                                          BH, N, scale, *bm, L)
+                  : launch<D, false, true>(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv,
+                                           BH, N, scale, *bm, L);
+  return causal ? launch<D, true, false>(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv, BH,
+                                         N, scale, none, L)
+                : launch<D, false, false>(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv,
+                                          BH, N, scale, none, L);
 }
 
 }  // namespace bwd
 
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tdo, const float* dvec, const float* lse2,
-                             void* dq, void* dk, void* dv, int BH, int N, int d, float scale,
-                             int causal, const BlockMaskArg* bm, const Launch& L) {
+                             const CUtensorMap& tdo, const void* o, const void* dO,
+                             const float* lse, float* dvec, float* lse2, void* dq, void* dk,
+                             void* dv, int BH, int N, int d, float scale, int causal,
+                             const BlockMaskArg* bm, const Launch& L) {
   switch (d) {
     case 64:
-      return bwd::launch_d<64>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale, causal, bm,
-                               L);
+      return bwd::launch_d<64>(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv, BH, N, scale,
+                               causal, bm, L);
     case 80:
-      return bwd::launch_d<80>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale, causal, bm,
-                               L);
+      return bwd::launch_d<80>(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv, BH, N, scale,
+                               causal, bm, L);
     case 128:
-      return bwd::launch_d<128>(tq, tk, tv, tdo, dvec, lse2, dq, dk, dv, BH, N, scale, causal,
-                                bm, L);
+      return bwd::launch_d<128>(tq, tk, tv, tdo, o, dO, lse, dvec, lse2, dq, dk, dv, BH, N,
+                                scale, causal, bm, L);
     default:
       return cudaErrorInvalidValue;
   }

@@ -21,7 +21,9 @@
 //   warp 8      TMA producer: both Q tiles of an item, then K_j and V_j into
 //               separate shared-memory rings; each K/V tile serves both Q
 //               tiles (half the K/V traffic per FLOP of a one-tile CTA).  It
-//               requests the next item once the current item's loads are out.
+//               requests the next item as soon as it starts the current one,
+//               so the next item's loads follow the current item's without a
+//               gap.
 //   warp 9      TMEM allocator and MMA issuer (one elected lane), alternating
 //               between the tiles: O_A += P_A V_j, S_A = Q_A K_{j+1}^T,
 //               O_B += P_B V_j, S_B = Q_B K_{j+1}^T, so the tensor core works
@@ -30,7 +32,11 @@
 //               per query row (= TMEM lane), base-2 domain, lazy rescaling
 //               (the reference max moves, and O and l are rescaled in TMEM,
 //               only when the row max grew by more than 2^8; exponents stay
-//               <= 8).  They also run their tile's epilogue (O / l, LSE).
+//               <= 8).  They also run their tile's epilogue (O / l, LSE):
+//               each warp writes its 32 rows of O, 64 columns at a time,
+//               into its own 4 KB swizzled staging buffer and one lane
+//               stores it with TMA (whole rows per transfer instead of one
+//               16-byte piece of 32 different rows per store instruction).
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+d),
 // O_B [384,384+d).  S of a tile is single-buffered: S_X(j+1) is issued after
 // O_X += P_X(j) V_j, so when the softmax sees S_X(j+1) the previous P V has
@@ -79,7 +85,9 @@ struct Cfg {
   static constexpr int Q_OFF = 0;           // [2] tiles A, B
   static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + NST * TILE;
-  static constexpr int BAR_OFF = V_OFF + NST * TILE;
+  static constexpr int STG_OFF = V_OFF + NST * TILE;  // [8 softmax warps] 4 KB O staging
+  static constexpr int STG = 4096;                     // 32 rows x 64 bf16 columns
+  static constexpr int BAR_OFF = STG_OFF + 8 * STG;
   static constexpr int NBAR = 2 + 4 * NST + 6 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
   static constexpr int SMEM = MISC_OFF + 48 + 1024;    // + slack for 1 KB alignment
@@ -205,7 +213,8 @@ __device__ __forceinline__ void split_plan(int idx, int n_t, int BH, int group,
 template <int D, bool CAUSAL, bool BS, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               __nv_bfloat16* __restrict__ out,
                float* __restrict__ lse, int N, int BH, int group, float scale_log2,
                const uint8_t* __restrict__ bmask, int mask_heads, int H, SplitKv sk,
                WaitCtl ctl) {
@@ -326,6 +335,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           idx = clc_result_x(nxt_resp + 16 * sl);
           if (idx < 0) break;
         }
+        // Ask for item i + 1 right away: its answer is then at hand when
+        // this item's last loads are out, and the next Q can follow them.
+        {
+          const int sl1 = (i + 1) & 1;
+          const uint32_t u1 = static_cast<uint32_t>(i >> 1);
+          if (u1 > 0 && !wait(nxt_empty + sl1, (u1 - 1) & 1)) break;
+          if (leader) {
+            mbar_arrive_expect_tx(nxt_full + sl1, 16);
+            clc_try_cancel(nxt_resp + 16 * sl1, nxt_full + sl1);
+          }
+          sync();
+          nxt_pending = sl1;
+          nxt_pending_par = u1 & 1;
+        }
         int bh, pair, n_x[2];
         ItemTiles<CAUSAL> tiles;
         int t0 = 0;  // first key tile of a split-KV item
@@ -382,17 +405,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
         }
-        // Ask for the next item now, while this one's MMAs and softmax run.
-        const int sl1 = (i + 1) & 1;
-        const uint32_t u1 = static_cast<uint32_t>(i >> 1);
-        if (u1 > 0 && !wait(nxt_empty + sl1, (u1 - 1) & 1)) break;
-        if (leader) {
-          mbar_arrive_expect_tx(nxt_full + sl1, 16);
-          clc_try_cancel(nxt_resp + 16 * sl1, nxt_full + sl1);
-        }
-        sync();
-        nxt_pending = sl1;
-        nxt_pending_par = u1 & 1;
       }
       if (*abort && leader) {
         // Let every copy and request this CTA started land before shared
@@ -526,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t col_s = x * kBN;
     const uint32_t col_o = 256 + x * kBN;
+
     uint32_t s_base = 0;  // s_full / o_done phases of this tile before the current item
     bool ok = true;
     int idx = 0;
@@ -703,21 +716,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (valid) sk.part_lse[prow] = lse_row;
         } else {
-          uint4* orow =
-              reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + q_idx) * D);
+          // O rows of this warp: 64 columns per TMA store (columns past d
+          // and rows past N are not written by the store).
+          // This warp's staging buffer (1 KB aligned: the 128-byte swizzle
+          // pattern repeats every 8 rows): row `lane`, 16-byte chunk c at
+          // chunk c ^ (lane % 8) of the row.  Its previous store must have
+          // read it first.
+          const int row0 = qt_x * kBM + (warp & 3) * 32;
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t o16[16];
-            tmem_ld16(lane_base + col_o + c * 16, o16);
-            tmem_wait_ld();
-            uint32_t pkd[8];
+          for (int b = 0; b < C::NB; ++b) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+            const uint32_t rowa = sbase + C::STG_OFF + warp * C::STG + lane * 128;
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              pkd[e] = pack_bf16(__uint_as_float(o16[2 * e]) * inv_l,
-                                 __uint_as_float(o16[2 * e + 1]) * inv_l);
-            if (valid) {
-              orow[2 * c] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
-              orow[2 * c + 1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+            for (int hf = 0; hf < 4; ++hf) {  // 16 columns = 2 chunks at a time
+              uint32_t t[16];
+              tmem_ld16(lane_base + col_o + 64 * b + 16 * hf, t);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c4 = 0; c4 < 2; ++c4) {
+                const int c = 2 * hf + c4, e0 = 8 * c4;
+                st_shared_v4(rowa + ((c ^ (lane & 7)) << 4),
+                             pack_bf16(__uint_as_float(t[e0 + 0]) * inv_l,
+                                       __uint_as_float(t[e0 + 1]) * inv_l),
+                             pack_bf16(__uint_as_float(t[e0 + 2]) * inv_l,
+                                       __uint_as_float(t[e0 + 3]) * inv_l),
+                             pack_bf16(__uint_as_float(t[e0 + 4]) * inv_l,
+                                       __uint_as_float(t[e0 + 5]) * inv_l),
+                             pack_bf16(__uint_as_float(t[e0 + 6]) * inv_l,
+                                       __uint_as_float(t[e0 + 7]) * inv_l));
+              }
+            }
+            fence_async_shared();
+            __syncwarp();
+            if (lane == 0 && row0 < N) {
+              tma_store_3d(&tm_o, smem + C::STG_OFF + warp * C::STG, 64 * b, row0, bh);
+              bulk_commit();
             }
           }
           if (valid) lse[static_cast<size_t>(bh) * N + q_idx] = lse_row;
@@ -730,6 +764,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       s_base += static_cast<uint32_t>(n_kv);
     }
+    // Shared memory must outlive the O stores that read it.
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -741,9 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, bool CAUSAL, bool BS, bool SPLIT>
-cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                   float* lse, int BH, int N, float scale, const BlockMaskArg& bm,
-                   const SplitKv& sk, const Launch& L) {
+cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const CUtensorMap& to, void* o, float* lse, int BH, int N, float scale,
+                   const BlockMaskArg& bm, const SplitKv& sk, const Launch& L) {
   using C = Cfg<D>;
   static bool configured = false;
   if (!configured) {
@@ -776,49 +813,52 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   WaitCtl ctl{L.status, L.limit_ns};
   fwd_kernel<D, CAUSAL, BS, SPLIT>
       <<<static_cast<unsigned>(blocks), kThreads, C::SMEM, L.stream>>>(
-          tq, tk, tv, static_cast<__nv_bfloat16*>(o), lse, N, BH, group, scale_log2, bm.mask,
+          tq, tk, tv, to, static_cast<__nv_bfloat16*>(o), lse, N, BH, group, scale_log2, bm.mask,
           bm.mask_heads, bm.H, sk, ctl);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                     void* o, float* lse, int BH, int N, float scale, int causal,
-                     const BlockMaskArg* bm, const Launch& L) {
+                     const CUtensorMap& to, void* o, float* lse, int BH, int N, float scale,
+                     int causal, const BlockMaskArg* bm, const Launch& L) {
   const BlockMaskArg none{nullptr, 1, 1};
   const SplitKv dense{N, 0, 1, (N + kBN - 1) / kBN, nullptr, nullptr};
   if (bm && bm->mask)
-    return causal ? launch<D, true, true, false>(tq, tk, tv, o, lse, BH, N, scale, *bm, dense, L)
-                  : launch<D, false, true, false>(tq, tk, tv, o, lse, BH, N, scale, *bm, dense,
-                                                  L);
-  return causal ? launch<D, true, false, false>(tq, tk, tv, o, lse, BH, N, scale, none, dense, L)
-                : launch<D, false, false, false>(tq, tk, tv, o, lse, BH, N, scale, none, dense,
-                                                 L);
+    return causal ? launch<D, true, true, false>(tq, tk, tv, to, o, lse, BH, N, scale, *bm, dense,
+                                                 L)
+                  : launch<D, false, true, false>(tq, tk, tv, to, o, lse, BH, N, scale, *bm,
+                                                  dense, L);
+  return causal ? launch<D, true, false, false>(tq, tk, tv, to, o, lse, BH, N, scale, none, dense,
+                                                L)
+                : launch<D, false, false, false>(tq, tk, tv, to, o, lse, BH, N, scale, none,
+                                                 dense, L);
 }
 
 template <int D>
 cudaError_t launch_split_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            int BH, int Nq, float scale, int causal, const SplitKv& sk,
                            const Launch& L) {
+  // Split launches write fp32 partials with plain stores: the O map is unused.
   const BlockMaskArg none{nullptr, 1, 1};
-  return causal ? launch<D, true, false, true>(tq, tk, tv, nullptr, nullptr, BH, Nq, scale, none,
-                                               sk, L)
-                : launch<D, false, false, true>(tq, tk, tv, nullptr, nullptr, BH, Nq, scale, none,
-                                                sk, L);
+  return causal ? launch<D, true, false, true>(tq, tk, tv, tq, nullptr, nullptr, BH, Nq, scale,
+                                               none, sk, L)
+                : launch<D, false, false, true>(tq, tk, tv, tq, nullptr, nullptr, BH, Nq, scale,
+                                                none, sk, L);
 }
 
 }  // namespace fwd
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             void* o, float* lse, int BH, int N, int d, float scale, int causal,
-                             const BlockMaskArg* bm, const Launch& L) {
+                             const CUtensorMap& to, void* o, float* lse, int BH, int N, int d,
+                             float scale, int causal, const BlockMaskArg* bm, const Launch& L) {
   switch (d) {
     case 64:
-      return fwd::launch_d<64>(tq, tk, tv, o, lse, BH, N, scale, causal, bm, L);
+      return fwd::launch_d<64>(tq, tk, tv, to, o, lse, BH, N, scale, causal, bm, L);
     case 80:
-      return fwd::launch_d<80>(tq, tk, tv, o, lse, BH, N, scale, causal, bm, L);
+      return fwd::launch_d<80>(tq, tk, tv, to, o, lse, BH, N, scale, causal, bm, L);
     case 128:
-      return fwd::launch_d<128>(tq, tk, tv, o, lse, BH, N, scale, causal, bm, L);
+      return fwd::launch_d<128>(tq, tk, tv, to, o, lse, BH, N, scale, causal, bm, L);
     default:
       return cudaErrorInvalidValue;
   }

@@ -28,6 +28,7 @@ enum WaitSite : int {
   kSiteBwdDq = 0x204,
   kSiteBwdEpilogue = 0x205,
   kSiteBwdDrain = 0x206,
+  kSiteBwdSmem = 0x207,  // dynamic shared memory base needed more alignment slack than left
   kSiteSelfTest = 0x7e57,
 };
 
@@ -75,10 +76,12 @@ struct SplitKv {
 
 // --- bf16 tensor-core path (fa_fwd_sm100.cu, fa_bwd_sm100.cu) -------------
 // Tensor maps describe a [BH, N, d] bf16 tensor as 3-D {d, N, BH} with a
-// {64, 128, 1} box and 128-byte swizzle.
+// {64, 128, 1} box (loads) or a {64, 32, 1} box (the forward's O stores,
+// `to`) and 128-byte swizzle.
+constexpr int kStoreBoxRows = 32;
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             void* o, float* lse, int BH, int N, int d, float scale, int causal,
-                             const BlockMaskArg* bm, const Launch& L);
+                             const CUtensorMap& to, void* o, float* lse, int BH, int N, int d,
+                             float scale, int causal, const BlockMaskArg* bm, const Launch& L);
 
 // Split-KV forward: tq has N_q rows per head, tk / tv N_k (sk.Nk) rows.
 cudaError_t launch_fwd_splitkv_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
@@ -91,15 +94,18 @@ cudaError_t launch_fwd_splitkv_sm100(const CUtensorMap& tq, const CUtensorMap& t
 cudaError_t launch_splitkv_combine(const float* part_o, const float* part_lse, void* o,
                                    float* lse, int n_split, int rows, int d, const Launch& L);
 
-// Backward: the dK/dV kernel then the dQ kernel, both in stream order.
-// dvec and lse2 are the preprocess outputs ([BH, Np] fp32, Np = N rounded up
-// to 128); dq, dk, dv are bf16 [BH, N, d] outputs.
+// Backward: the dQ kernel then the dK/dV kernel, in stream order.  The dQ
+// kernel computes the row statistics D = rowsum(dO o O) and LSE2 = LSE log2(e)
+// from o, dO (bf16 [BH, N, d]) and lse and writes them to dvec and lse2
+// ([BH, Np] fp32, Np = N rounded up to 128; D = 0 and LSE2 = +inf past N),
+// where the dK/dV kernel reads them; dq, dk, dv are bf16 [BH, N, d] outputs.
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tdo, const float* dvec, const float* lse2,
-                             void* dq, void* dk, void* dv, int BH, int N, int d, float scale,
-                             int causal, const BlockMaskArg* bm, const Launch& L);
+                             const CUtensorMap& tdo, const void* o, const void* dO,
+                             const float* lse, float* dvec, float* lse2, void* dq, void* dk,
+                             void* dv, int BH, int N, int d, float scale, int causal,
+                             const BlockMaskArg* bm, const Launch& L);
 
-// --- helpers shared by both dtypes (fa_simt.cu) ---------------------------
+// --- fp32 path helper (fa_simt.cu) -----------------------------------------
 // D = rowsum(dO o O) (fp32, padded rows = 0) and, when lse2 is non-null,
 // lse2 = LSE * log2(e) (padded rows = +inf).
 cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse, float* dvec,

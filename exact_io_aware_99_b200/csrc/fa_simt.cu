@@ -1,8 +1,8 @@
 // fa_simt.cu -- CUDA-core kernels of the attention library:
 //   * the fp32 forward and backward (fp32 FMA throughout, for accuracy
 //     checks at small sizes; TF32 tensor cores cannot hold 1e-5),
-//   * the backward preprocess shared by both dtypes
-//     (D = rowsum(dO o O) and the base-2 LSE, padded to whole 128-row tiles),
+//   * the fp32 backward's preprocess (D = rowsum(dO o O), padded to whole
+//     128-row tiles; the bf16 backward computes D in its dQ kernel),
 //   * the bounded-wait self test.
 //
 // The forward follows the blocked algorithm of the "FlashAttention-2" review

@@ -126,10 +126,11 @@ FA_API size_t fa_backward_workspace_size(int B, int H, int N, int d);
  *                   not matter and are clobbered.  Two calls that overlap on
  *                   the GPU must not share one workspace.
  *   Other arguments as in fa_forward (same scale and causal as the forward).
- * Launches three kernels in stream order: the preprocess (D and the base-2
- * LSE), the dK/dV kernel and the dQ kernel.  dQ is computed by its own kernel
- * (it recomputes S and dP per query tile), so no atomics are used and the
- * result is bitwise reproducible.
+ * Launches two kernels in stream order: the dQ kernel (which also writes the
+ * row statistics D = rowsum(dO o O) and the base-2 LSE into the workspace)
+ * and the dK/dV kernel.  dQ is computed by its own kernel (it recomputes S
+ * and dP per query tile), so no atomics are used and the result is bitwise
+ * reproducible.
  */
 FA_API fa_status fa_backward(const void* q, const void* k, const void* v,
                       const void* o, const void* dO, const float* lse,
