@@ -9,6 +9,7 @@ Low-level entry points (same names as the C ABI): ``fa_forward``,
 ``fa_backward_noalloc``, ``fa_forward_blocksparse``, ``fa_backward_blocksparse``,
 ``fa_forward_splitkv``, ``fa_splitkv_default_splits``, ``fa_splitkv_workspace_size``,
 ``fa_backward_workspace_size``, ``fa_forward_fp8``, ``fa_quantize_fp8``,
+``fa_set_forward_key_tile``, ``fa_forward_key_tile``,
 ``fa_status_string``, ``fa_device_status``, ``fa_set_wait_timeout_ns``,
 ``fa_selftest_wait_timeout``.
 
@@ -35,6 +36,7 @@ _NATIVE = {
     "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_forward_blocksparse",
     "fa_backward_blocksparse", "fa_forward_splitkv", "fa_splitkv_default_splits",
     "fa_splitkv_workspace_size", "fa_forward_fp8", "fa_quantize_fp8",
+    "fa_set_forward_key_tile", "fa_forward_key_tile",
 }
 _API = {"attention_forward", "attention_backward", "attention_decode",
         "attention_forward_fp8", "quantize_fp8"}

@@ -32,7 +32,7 @@ EXPORTS = (
     "fa_set_wait_timeout_ns", "fa_selftest_wait_timeout", "fa_backward_noalloc",
     "fa_forward_blocksparse", "fa_backward_blocksparse", "fa_forward_splitkv",
     "fa_splitkv_default_splits", "fa_splitkv_workspace_size", "fa_forward_fp8",
-    "fa_quantize_fp8",
+    "fa_quantize_fp8", "fa_set_forward_key_tile", "fa_forward_key_tile",
 )
 
 # Size of the library's built-in scratch array used by fa_backward_noalloc.
@@ -91,6 +91,10 @@ def _load() -> ctypes.CDLL:
     lib.fa_forward_fp8.restype = I
     lib.fa_quantize_fp8.argtypes = [P, I, S, P, P, P]
     lib.fa_quantize_fp8.restype = I
+    lib.fa_set_forward_key_tile.argtypes = [I]
+    lib.fa_set_forward_key_tile.restype = I
+    lib.fa_forward_key_tile.argtypes = [I, I, I]
+    lib.fa_forward_key_tile.restype = I
     return lib
 
 
@@ -174,6 +178,17 @@ def fa_device_status(reset: bool = True):
 
 def fa_set_wait_timeout_ns(ns: int) -> None:
     _lib.fa_set_wait_timeout_ns(int(ns))
+
+
+def fa_set_forward_key_tile(keys: int, check=True) -> int:
+    """Force the dense bf16 forward's key-tile size (64 or 128) for every
+    later call, or restore the built-in table (0)."""
+    return _check(_lib.fa_set_forward_key_tile(int(keys)), "fa_set_forward_key_tile", check)
+
+
+def fa_forward_key_tile(d: int, N: int, causal: bool) -> int:
+    """Key-tile size the dense bf16 forward uses for this shape (0: unsupported)."""
+    return int(_lib.fa_forward_key_tile(int(d), int(N), int(bool(causal))))
 
 
 def fa_selftest_wait_timeout(stream=None, check=True) -> int:

@@ -21,6 +21,24 @@ __device__ int g_fa_status = 0;
 
 constexpr unsigned long long kDefaultLimitNs = 2000000000ull;
 std::atomic<unsigned long long> g_limit_ns{kDefaultLimitNs};
+// Key-tile size of the dense bf16 forward: 0 = the built-in table, else 64
+// or 128 (fa_set_forward_key_tile).
+std::atomic<int> g_fwd_key_tile{0};
+
+// Key-tile size of the dense bf16 forward for a problem: the 64-key kernel
+// (two score buffers per query tile) or the 128-key kernel.  The table is the
+// measured winner on B200 (both kernels timed on the same inputs, L2 flushed,
+// B H N = 262144): the 64-key kernel is ahead only for short causal problems,
+// where most key steps are diagonal or ragged and its finer key tiles skip
+// more masked work (d = 128 causal: +4 % at N = 128 and 256, even at 512;
+// d = 64 causal: +6 % at N = 512); elsewhere its twice as many, half as wide
+// score MMAs cost 6-25 %.
+int forward_key_tile(int d, int N, int causal) {
+  const int forced = g_fwd_key_tile.load(std::memory_order_relaxed);
+  if (forced == 64 || forced == 128) return forced;
+  if (!causal) return 128;
+  return N <= (d == 64 ? 512 : 256) ? 64 : 128;
+}
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
@@ -175,6 +193,17 @@ void fa_set_wait_timeout_ns(unsigned long long ns) {
   g_limit_ns.store(ns ? ns : kDefaultLimitNs, std::memory_order_relaxed);
 }
 
+fa_status fa_set_forward_key_tile(int keys) {
+  if (keys != 0 && keys != 64 && keys != 128) return FA_ERR_INVALID_ARG;
+  g_fwd_key_tile.store(keys, std::memory_order_relaxed);
+  return FA_OK;
+}
+
+int fa_forward_key_tile(int d, int N, int causal) {
+  if (N < 1 || (d != 64 && d != 80 && d != 128)) return 0;
+  return forward_key_tile(d, N, causal ? 1 : 0);
+}
+
 fa_status fa_device_status(int reset, int* site) {
   fa::Launch L;
   fa_status st = device_context(nullptr, &L);
@@ -222,12 +251,14 @@ fa_status fa_forward_ex(const void* q, const void* k, const void* v, void* o, fl
   } else {
     st = get_encoder();
     if (st != FA_OK) return st;
+    const int kt = forward_key_tile(d, N, cz);
     CUtensorMap tq, tk, tv, to;
     if ((st = make_map(&tq, q, BH, N, d)) != FA_OK) return st;
-    if ((st = make_map(&tk, k, BH, N, d)) != FA_OK) return st;
-    if ((st = make_map(&tv, v, BH, N, d)) != FA_OK) return st;
+    if ((st = make_map(&tk, k, BH, N, d, kt)) != FA_OK) return st;
+    if ((st = make_map(&tv, v, BH, N, d, kt)) != FA_OK) return st;
     if ((st = make_map(&to, o, BH, N, d, fa::kStoreBoxRows)) != FA_OK) return st;
-    e = fa::launch_fwd_sm100(tq, tk, tv, to, o, lse, BH, N, d, scale, cz, nullptr, L);
+    e = kt == 64 ? fa::launch_fwd64_sm100(tq, tk, tv, to, lse, BH, N, d, scale, cz, L)
+                 : fa::launch_fwd_sm100(tq, tk, tv, to, o, lse, BH, N, d, scale, cz, nullptr, L);
   }
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }

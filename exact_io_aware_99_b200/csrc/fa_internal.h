@@ -83,6 +83,13 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
                              const CUtensorMap& to, void* o, float* lse, int BH, int N, int d,
                              float scale, int causal, const BlockMaskArg* bm, const Launch& L);
 
+// Forward with 64-key tiles and two score buffers per query tile
+// (fa_fwd64_sm100.cu); tk and tv have {64, 64, 1} boxes, tq {64, 128, 1},
+// to {64, 32, 1}.  Dense only (no block mask, no split).
+cudaError_t launch_fwd64_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const CUtensorMap& to, float* lse, int BH, int N, int d,
+                               float scale, int causal, const Launch& L);
+
 // Split-KV forward: tq has N_q rows per head, tk / tv N_k (sk.Nk) rows.
 cudaError_t launch_fwd_splitkv_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                      const CUtensorMap& tv, int BH, int Nq, int d, float scale,

@@ -329,6 +329,26 @@ FA_API fa_status fa_device_status(int reset, int* site);
 FA_API void fa_set_wait_timeout_ns(unsigned long long ns);
 
 /*
+ * Key-tile size of the dense bf16 forward (fa_forward, fa_forward_ex with
+ * FA_BF16).  The block sizes B_r x B_c of the tiled algorithm are left to be
+ * tuned per GPU ("FlashAttention-2: Faster Attention with Better Parallelism
+ * and Work Partitioning" review page, implementation-cost answer, section
+ * (2), and auto-tuning answer, section 1 (1), which lists candidate sizes).
+ * The library has two forward kernels with 128-row query tiles: one with
+ * 128-key tiles and one with 64-key tiles and two score buffers per query
+ * tile, and a built-in table that picks one from (d, N, causal).
+ *
+ * fa_set_forward_key_tile(keys): 0 restores the table; 64 or 128 forces that
+ * kernel for every later call (a process-wide setting, e.g. for measuring
+ * both); anything else is FA_ERR_INVALID_ARG.  Block-sparse and split-KV
+ * forwards always use 128-key tiles.
+ * fa_forward_key_tile(d, N, causal): the key-tile size the next dense bf16
+ * forward of that shape would use (64 or 128), 0 for an unsupported shape.
+ */
+FA_API fa_status fa_set_forward_key_tile(int keys);
+FA_API int fa_forward_key_tile(int d, int N, int causal);
+
+/*
  * fa_selftest_wait_timeout -- failure-detection self test: launches one
  * 32-thread block that waits on a barrier nothing ever completes, under the
  * current time limit; the wait gives up, records its site code (0x7e57) in

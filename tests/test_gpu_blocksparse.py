@@ -98,16 +98,22 @@ def test_band_with_global_columns_non_causal():
 
 
 def test_all_blocks_on_matches_dense_path():
+    # the block-sparse forward is the 128-key kernel with a mask: with every
+    # block on it must reproduce the dense 128-key kernel bit for bit
     m = fa()
     x = workloads.random_case(1, 2, 513, 128, 960)
     q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
     nt = 5
     bm = torch.ones((nt, nt), dtype=torch.uint8)
-    for causal in (False, True):
-        o1, l1 = m.attention_forward(q, k, v, causal=causal, block_mask=bm)
-        o2, l2 = m.attention_forward(q, k, v, causal=causal)
-        torch.cuda.synchronize()
-        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    m.fa_set_forward_key_tile(128)
+    try:
+        for causal in (False, True):
+            o1, l1 = m.attention_forward(q, k, v, causal=causal, block_mask=bm)
+            o2, l2 = m.attention_forward(q, k, v, causal=causal)
+            torch.cuda.synchronize()
+            assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    finally:
+        m.fa_set_forward_key_tile(0)
 
 
 def test_everything_hidden_gives_zeros():

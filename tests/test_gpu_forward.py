@@ -16,6 +16,16 @@ def case(B, H, N, d, seed, dtype=torch.bfloat16, std=1.0):
     return workloads.random_case(B, H, N, d, seed, dtype=dtype, grad=False, std=std)
 
 
+@pytest.fixture(params=[128, 64], ids=["keys128", "keys64"])
+def key_tile(request):
+    """Run the test on both dense bf16 forward kernels (128-key tiles, and
+    64-key tiles with two score buffers per query tile)."""
+    import exact_io_aware_99_b200 as fa
+    fa.fa_set_forward_key_tile(request.param)
+    yield request.param
+    fa.fa_set_forward_key_tile(0)
+
+
 # ------------------------------------------------------------------ fp32 path
 
 def test_fp32_workload_full_size():
@@ -36,19 +46,19 @@ def test_fp32_odd_sizes(N, d, causal):
 @pytest.mark.parametrize("d", [64, 80, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 7, 127, 128, 129, 300, 1000])
-def test_bf16_small_shapes(N, d, causal):
+def test_bf16_small_shapes(N, d, causal, key_tile):
     x = case(1, 2, N, d, 100 * d + N + causal)
     check_forward(x["q"], x["k"], x["v"], 1 / math.sqrt(d), causal)
 
 
 @pytest.mark.parametrize("d", [64, 128])
-def test_bf16_several_heads_and_batches(d):
+def test_bf16_several_heads_and_batches(d, key_tile):
     x = case(3, 5, 513, d, 77 + d)
     check_forward(x["q"], x["k"], x["v"], 1 / math.sqrt(d), True)
 
 
 @pytest.mark.parametrize("causal", [False, True])
-def test_growing_scores_force_a_rescale_every_tile(causal):
+def test_growing_scores_force_a_rescale_every_tile(causal, key_tile):
     # Score of key j is 0.05 j: the row max grows by 6.4 (> 8 in base 2) per
     # 128-key tile, so the running output is rescaled on every tile.
     N, d = 1024, 128
@@ -60,7 +70,7 @@ def test_growing_scores_force_a_rescale_every_tile(causal):
     check_forward(q.bfloat16(), k.bfloat16(), v.bfloat16(), 1.0, causal)
 
 
-def test_identical_keys_give_the_mean_of_values():
+def test_identical_keys_give_the_mean_of_values(key_tile):
     N, d = 384, 64
     x = case(1, 1, N, d, 9)
     k = x["k"][:, :, :1].expand(1, 1, N, d).contiguous()
@@ -71,7 +81,7 @@ def test_identical_keys_give_the_mean_of_values():
     assert float((o[0, 0].double().cpu() - means).abs().max()) <= TOL_O_BF16
 
 
-def test_large_magnitude_scores():
+def test_large_magnitude_scores(key_tile):
     # std 3 inputs: scores with std 9 (very peaked rows) and |V| up to ~13.
     # The 1e-2 bound is stated for unit-variance inputs; here the bound is
     # derived from the arithmetic: P is rounded to bf16 before P V (relative
@@ -83,7 +93,7 @@ def test_large_magnitude_scores():
                   tol_o=(2.0 ** -8 + 2.0 ** -9) * vmax)
 
 
-def test_outputs_beyond_n_are_untouched():
+def test_outputs_beyond_n_are_untouched(key_tile):
     # The kernel must not write rows >= N of O or LSE (ragged last tile).
     N, d = 200, 64
     x = case(1, 1, N, d, 3)
@@ -106,8 +116,19 @@ def test_outputs_beyond_n_are_untouched():
 
 @pytest.mark.parametrize("name", ["fwd_d64", "causal_d128", "long_d128", "gpt3_d80"])
 def test_full_size_workload_forward(name):
+    # the kernel the built-in key-tile table picks for this shape
     w = workloads.WORKLOADS[name]
     x = workloads.make_inputs(w, with_grad_out=False)
     heads = (None if name == "fwd_d64"
              else l2_group_heads(w.B, w.H, w.N, w.d, w.causal))
     check_forward(x["q"], x["k"], x["v"], w.scale, w.causal, heads=heads)
+
+
+@pytest.mark.parametrize("name", ["causal_d128", "gpt3_d80"])
+def test_full_size_workload_forward_both_kernels(name, key_tile):
+    # both kernels on the full-size workloads, whatever the table would pick
+    w = workloads.WORKLOADS[name]
+    x = workloads.make_inputs(w, with_grad_out=False)
+    check_forward(x["q"], x["k"], x["v"], w.scale, w.causal,
+                  heads=l2_group_heads(w.B, w.H, w.N, w.d, w.causal))
+

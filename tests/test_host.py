@@ -259,3 +259,26 @@ def test_fp8_step_counts_only_the_forward():
     assert b == 0.0
     assert f == perf.fwd_flops(4, 16, 4096, 128, True)
     assert abs(f - 274.9e9) < 0.1e9
+
+
+def test_forward_key_tile_table_and_override():
+    # host-side logic only: the table picks the 64-key kernel for short causal
+    # problems, the override forces either kernel, bad sizes are rejected
+    m = _lib()
+    assert m.fa_forward_key_tile(128, 256, True) == 64
+    assert m.fa_forward_key_tile(128, 257, True) == 128
+    assert m.fa_forward_key_tile(80, 200, True) == 64
+    assert m.fa_forward_key_tile(64, 512, True) == 64
+    assert m.fa_forward_key_tile(64, 513, True) == 128
+    assert m.fa_forward_key_tile(128, 128, False) == 128
+    assert m.fa_forward_key_tile(96, 128, True) == 0
+    assert m.fa_forward_key_tile(128, 0, True) == 0
+    assert m.fa_set_forward_key_tile(7, check=False) == m.FA_ERR_INVALID_ARG
+    try:
+        m.fa_set_forward_key_tile(128)
+        assert m.fa_forward_key_tile(128, 256, True) == 128
+        m.fa_set_forward_key_tile(64)
+        assert m.fa_forward_key_tile(128, 16384, False) == 64
+    finally:
+        m.fa_set_forward_key_tile(0)
+    assert m.fa_forward_key_tile(128, 16384, False) == 128
