@@ -132,11 +132,14 @@ __device__ __forceinline__ int count_tiles(const Tiles& t) {
 }
 
 // Store one row of a tile from TMEM columns [taddr, taddr + D) (fp32, times
-// `mul`) to global memory as bf16, 16 columns per step; the steps alternate
-// between the two softmax warpgroups (h = 0, 1).
+// `mul`) to global memory as bf16, 16 columns (32 bytes) per step; the steps
+// alternate between the two softmax warpgroups (h = 0, 1).  Every thread
+// writes its own row, so a warp's store touches 32 rows: with `wide` (the
+// tensor 32-byte aligned, hence every 32-byte piece of a row) each piece is
+// one 32-byte store, a whole L2 sector, instead of two 16-byte halves.
 template <int D>
 __device__ __forceinline__ void store_row_bf16(uint32_t taddr, float mul, __nv_bfloat16* row,
-                                               bool valid, int h) {
+                                               bool valid, int h, bool wide) {
 #pragma unroll
   for (int c = 0; c < D / 16; ++c) {
     if ((c & 1) != h) continue;
@@ -148,9 +151,13 @@ __device__ __forceinline__ void store_row_bf16(uint32_t taddr, float mul, __nv_b
     for (int e = 0; e < 8; ++e)
       pk[e] = pack_bf16(__uint_as_float(v16[2 * e]) * mul, __uint_as_float(v16[2 * e + 1]) * mul);
     if (valid) {
-      uint4* dst = reinterpret_cast<uint4*>(row + c * 16);
-      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      if (wide) {
+        st_global_v8(row + c * 16, pk);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(row + c * 16);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
     }
   }
 }
@@ -265,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dk,
                     __nv_bfloat16* __restrict__ dv, int N, int BH, int group, float scale,
                     float scale_log2, const uint8_t* __restrict__ bmask, int mask_heads, int H,
-                    WaitCtl ctl) {
+                    bool wide, WaitCtl ctl) {
   using C = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   {
@@ -692,8 +699,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++kv_items;
       tc_fence_after();
       const size_t row = (static_cast<size_t>(bh) * N + k_idx) * D;
-      store_row_bf16<D>(lane_base + kKvColDV, 1.f, dv + row, key_ok, h);
-      store_row_bf16<D>(lane_base + kKvColDK, scale, dk + row, key_ok, h);
+      store_row_bf16<D>(lane_base + kKvColDV, 1.f, dv + row, key_ok, h, wide);
+      store_row_bf16<D>(lane_base + kKvColDK, scale, dk + row, key_ok, h, wide);
       tc_fence_before();
       qbase += static_cast<uint32_t>(n_iter);
     }
@@ -743,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ dvec,
                   const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dq, int N, int BH,
                   int group, float scale, float scale_log2, const uint8_t* __restrict__ bmask,
-                  int mask_heads, int H, WaitCtl ctl) {
+                  int mask_heads, int H, bool wide, WaitCtl ctl) {
   using C = QCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -1114,7 +1121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++q_items;
       tc_fence_after();
       store_row_bf16<D>(lane_base + kQColDQ, scale, dq + (static_cast<size_t>(bh) * N + q_idx) * D,
-                        q_idx < N, h);
+                        q_idx < N, h, wide);
       tc_fence_before();
       kbase += static_cast<uint32_t>(n_kv);
     }
@@ -1224,17 +1231,21 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
       lse2, BH, N, n_t * kT);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // 32-byte row stores when every gradient tensor allows them (rows of
+  // 128, 160 or 256 bytes keep a 32-byte aligned base aligned).
+  const bool wide = ((reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) |
+                      reinterpret_cast<uintptr_t>(dv)) & 31u) == 0;
   bwd_dq_kernel<D, CAUSAL, BS>
       <<<static_cast<unsigned>(blocks), kThreads, QCfg<D>::SMEM, L.stream>>>(
           tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dq), N, BH, group, scale,
-          scale_log2, bm.mask, bm.mask_heads, bm.H, ctl);
+          scale_log2, bm.mask, bm.mask_heads, bm.H, wide, ctl);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bwd_dkdv_kernel<D, CAUSAL, BS>
       <<<static_cast<unsigned>(blocks), kThreads, KvCfg<D>::SMEM, L.stream>>>(
           tq, tk, tv, tdo, dvec, lse2, static_cast<__nv_bfloat16*>(dk),
           static_cast<__nv_bfloat16*>(dv), N, BH, group, scale, scale_log2, bm.mask,
-          bm.mask_heads, bm.H, ctl);
+          bm.mask_heads, bm.H, wide, ctl);
   return cudaGetLastError();
 }
 

@@ -219,8 +219,9 @@ FA_API fa_status fa_forward_splitkv(const void* q, const void* k, const void* v,
                                     float scale, int causal, int num_splits, void* workspace,
                                     size_t workspace_bytes, void* stream);
 
-/* Key splits for fa_forward_splitkv that give about four work items per SM
- * of the current device (1 .. ceil(N_k / 128)); 0 for invalid sizes. */
+/* Key splits for fa_forward_splitkv that give every SM of the current device
+ * about one work item (floor(SMs / items), clamped to 1 .. ceil(N_k / 128));
+ * 0 for invalid sizes. */
 FA_API int fa_splitkv_default_splits(int B, int H, int Nq, int Nk);
 
 /* Workspace bytes fa_forward_splitkv needs for these sizes and num_splits:

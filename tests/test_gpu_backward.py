@@ -57,3 +57,30 @@ def test_full_size_workload_backward(name):
     x = workloads.make_inputs(w)
     check_backward(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal,
                    heads=l2_group_heads(w.B, w.H, w.N, w.d, w.causal))
+
+
+def test_gradients_at_16_byte_aligned_addresses_match_the_32_byte_path():
+    # The gradient rows are written with 32-byte stores when dQ, dK and dV are
+    # 32-byte aligned and with 16-byte stores otherwise: both give the same bits.
+    import exact_io_aware_99_b200 as fa
+    from gpu_cases import gpu_forward
+    B, H, N, d = 1, 3, 300, 128
+    x = workloads.random_case(B, H, N, d, 4343)
+    o, lse = gpu_forward(x["q"], x["k"], x["v"], 1 / math.sqrt(d), True)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    n = B * H * N * d
+    wb = fa.fa_backward_workspace_size(B, H, N, d)
+    ws = torch.empty(wb, device="cuda", dtype=torch.uint8)
+    outs = []
+    for off in (0, 8):  # elements: 8 bf16 = 16 bytes
+        bufs = [torch.empty(n + 16, device="cuda", dtype=torch.bfloat16) for _ in range(3)]
+        g = [b_[off:off + n].view(B, H, N, d) for b_ in bufs]
+        assert (g[0].data_ptr() & 31) == (0 if off == 0 else 16)
+        fa.fa_backward(q, k, v, o, do, lse, g[0], g[1], g[2], B, H, N, d, 1 / math.sqrt(d),
+                       True, ws, wb)
+        torch.cuda.synchronize()
+        outs.append([t.clone() for t in g])
+    st, site = fa.fa_device_status(reset=True)
+    assert st == 0, f"device wait timed out at site {site:#x}"
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
