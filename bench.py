@@ -405,7 +405,7 @@ def run_ours(args, peaks, peak_kind):
                      "unit": "TFLOP/s", "frac": round(bwd_tf / peak, 4),
                      "traffic": traffic,
                      "algorithmic_bytes": perf.bwd_bytes(B, H, N, d)},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 4 * args.steps,
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                    "reasons": clk["reasons"], "samples": clk["samples"]},
         "e2e": e2e,
