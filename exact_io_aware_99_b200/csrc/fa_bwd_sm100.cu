@@ -670,6 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(lane_base + col_dp + kKvOffP, pk);
         tmem_wait_st();
         warp_arrive(p_full);
+        // dS^T = P^T o (dP^T - D), formed as P dP - P D on column pairs
+        // (two paired fp32 operations per pair).
         uint32_t dsk[32];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -677,12 +679,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; e += 4) {
             const float4 dv4 = *reinterpret_cast<const float4*>(dd + c * 32 + e);
             const uint32_t p01 = pk[c * 16 + e / 2], p23 = pk[c * 16 + e / 2 + 1];
-            const float d0 = bf16lo(p01) * (__uint_as_float(dpv[c][e + 0]) - dv4.x);
-            const float d1 = bf16hi(p01) * (__uint_as_float(dpv[c][e + 1]) - dv4.y);
-            const float d2 = bf16lo(p23) * (__uint_as_float(dpv[c][e + 2]) - dv4.z);
-            const float d3 = bf16hi(p23) * (__uint_as_float(dpv[c][e + 3]) - dv4.w);
-            dsk[c * 16 + e / 2] = pack_bf16(d0, d1);
-            dsk[c * 16 + e / 2 + 1] = pack_bf16(d2, d3);
+            const float2 pa = make_float2(bf16lo(p01), bf16hi(p01));
+            const float2 pb = make_float2(bf16lo(p23), bf16hi(p23));
+            const float2 ra = __ffma2_rn(pa, make_float2(__uint_as_float(dpv[c][e + 0]),
+                                                         __uint_as_float(dpv[c][e + 1])),
+                                         __fmul2_rn(pa, make_float2(-dv4.x, -dv4.y)));
+            const float2 rb = __ffma2_rn(pb, make_float2(__uint_as_float(dpv[c][e + 2]),
+                                                         __uint_as_float(dpv[c][e + 3])),
+                                         __fmul2_rn(pb, make_float2(-dv4.z, -dv4.w)));
+            dsk[c * 16 + e / 2] = pack_bf16(ra.x, ra.y);
+            dsk[c * 16 + e / 2 + 1] = pack_bf16(rb.x, rb.y);
           }
         }
         // dS^T -> the last 32 of this half's dP^T columns.
@@ -1100,13 +1106,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + col_dp, dpv[0]);
         tmem_ld32(lane_base + col_dp + 32, dpv[1]);
         tmem_wait_ld();
+        // dS = P o (dP - D), formed as P dP - P D on column pairs.
         uint32_t dsk[32];
+        const float2 nd2 = make_float2(-my_d, -my_d);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int c0 = 2 * c, c1 = 2 * c + 1;
-          const float d0 = p[c0] * (__uint_as_float(dpv[c0 >> 5][c0 & 31]) - my_d);
-          const float d1 = p[c1] * (__uint_as_float(dpv[c1 >> 5][c1 & 31]) - my_d);
-          dsk[c] = pack_bf16(d0, d1);
+          const float2 pp = make_float2(p[c0], p[c1]);
+          const float2 r = __ffma2_rn(pp, make_float2(__uint_as_float(dpv[c0 >> 5][c0 & 31]),
+                                                      __uint_as_float(dpv[c1 >> 5][c1 & 31])),
+                                      __fmul2_rn(pp, nd2));
+          dsk[c] = pack_bf16(r.x, r.y);
         }
         // dS -> the first 32 of this half's dP columns (already read).
         tmem_st32(lane_base + col_dp, dsk);
