@@ -6,9 +6,9 @@ oracle (exact attention of the dequantised inputs) does not do, so:
 
 * on inputs whose probabilities are exact E4M3 values
   (``workloads.fp8_exact_case``) the kernel must match the oracle up to the
-  bf16 rounding of O and the tensor core's accumulation: |err| <= 2^-8 |O|
-  + (2^-20 + (ceil(N/32) + 2) 2^-24) max|V|, the second term derived from the
-  MMA's accumulation window measured by a test below;
+  bf16 rounding of O (half an ulp, at most 2^-8 |O|) and the tensor core's
+  accumulation, (2^-20 + (ceil(N/32) + 2) 2^-24) max|V|, derived from the
+  MMA's accumulation window, which a test below measures;
 * on iid-normal inputs it must stay within ``oracle.fp8.p_rounding_bound``
   (the most rounding P to E4M3 can move each element) plus the same bf16 /
   fp32 allowance;
@@ -67,17 +67,30 @@ def accumulation_bound(n_keys):
     return 32 * 2.0 ** -WINDOW_BINADES + (n_steps + 2) * 2.0 ** -24
 
 
-def allowance(ro, vmax, n_keys):
-    """bf16 rounding of O (half an ulp is at most 2^-9 |O|, doubled) and the
+def half_ulp_bf16(x):
+    """Half the spacing of the bf16 grid at |x| (8 significant bits): the most
+    rounding to bf16 can move a value of that magnitude."""
+    a = np.maximum(np.abs(x), np.finfo(np.float32).tiny)
+    return np.exp2(np.floor(np.log2(a)) - 8.0)
+
+
+def allowance(ro, go, vmax, n_keys):
+    """Rounding O to bf16 (half an ulp at the larger of the reference and
+    the result, so a result that crossed a power of two is covered) plus the
     tensor core's accumulation of the E4M3 products of P V (derived above
-    from the measured window)."""
-    return 2.0 ** -8 * np.abs(ro) + accumulation_bound(n_keys) * vmax
+    from the measured window).  Returns (rounding part, accumulation part)."""
+    big = np.maximum(np.abs(ro), np.abs(go))
+    # the fp32 normalisation by 1/l (a reciprocal and a product) adds a few
+    # fp32 ulps of |O| before the bf16 rounding
+    return (half_ulp_bf16(big) + 2.0 ** -22 * big,
+            accumulation_bound(n_keys) * vmax)
 
 
 def compare(x, o, lse, scale, causal, heads=None, exact=False):
     B, H = x["q8"].shape[:2]
     pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
     worst = 0.0
+    worst_acc = 0.0  # share of the accumulation term used beyond rounding
     for b, h in pairs:
         q = dequantize(x["q8"][b, h], x["q_descale"])
         k = dequantize(x["k8"][b, h], x["k_descale"])
@@ -86,17 +99,19 @@ def compare(x, o, lse, scale, causal, heads=None, exact=False):
                          x["k_descale"], x["v_descale"], scale, causal)
         go, gl = np64(o[b, h]), np64(lse[b, h])
         assert np.all(np.isfinite(go)) and np.all(np.isfinite(gl))
-        tol = allowance(ro, float(np.abs(v).max()), ro.shape[0])
+        rnd, acc = allowance(ro, go, float(np.abs(v).max()), ro.shape[0])
         if not exact:
-            tol = tol + p_rounding_bound(q, k, v, scale, causal)
+            rnd = rnd + p_rounding_bound(q, k, v, scale, causal)
+        tol = rnd + acc
         err = np.abs(go - ro)
         bad = err > tol
         assert not bad.any(), (f"head ({b},{h}): {int(bad.sum())} elements outside the bound, "
                                f"worst excess {float((err - tol).max()):.3g}")
         worst = max(worst, float((err / tol).max()))
+        worst_acc = max(worst_acc, float((np.maximum(err - rnd, 0.0) / acc).max()))
         el = float(np.max(np.abs(gl - rl)))
         assert el <= TOL_LSE, f"LSE max abs err {el:.3g}"
-    print(f"worst |err| / allowed = {worst:.3g}")
+    print(f"worst |err| / allowed = {worst:.3g}; accumulation term used {worst_acc:.3g}")
     return worst
 
 
@@ -245,14 +260,14 @@ def test_mma_window_keeps_25_binades_below_the_group_max():
     # 2^-17 .. 2^-2 sharing that step.  Those at least 2^-25 of 2^16 (2^-9 and
     # up) must survive; O is exact attention up to bf16 rounding.
     m = fa()
-    N, d = 256, 16
+    N, d = 256, 64
     q = torch.zeros(1, 1, N, d)
     q[..., 0] = 1.0
     k = torch.zeros(1, 1, N, d)
     k[0, 0, 128:, 0] = -8.0
     k[0, 0, 128:130, 0] = 8.0
     v = torch.zeros(1, 1, N, d)
-    for c in range(d):
+    for c in range(16):
         v[0, 0, 128:, c] = 2.0 ** (-9 + c)
     v[0, 0, 128, :] = 256.0
     v[0, 0, 129, :] = -256.0
@@ -265,7 +280,7 @@ def test_mma_window_keeps_25_binades_below_the_group_max():
     torch.cuda.synchronize()
     l = 128 + 2 * 256 + 126 * 2.0 ** -8
     got = o[0, 0, 0].float().cpu().numpy()
-    for c in range(d):
+    for c in range(16):
         small = 2.0 ** (-8 - 9 + c)          # one small product
         if 16 - (-17 + c) > WINDOW_BINADES:  # outside the window: not asserted
             continue
