@@ -433,36 +433,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (c >= lim) s[c] = -INFINITY;
         }
-        float mx4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-        for (int c = 4; c < kBN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float mx = row_max(s);
         const float m_cand = fmaxf(m, mx * scale_log2);
         const bool grow = m_cand > m + kRescaleLog2;  // true on the first tile
-        const float alpha = grow ? ex2(m - m_cand) : 1.f;
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O_x must hold every earlier P V before it is rescaled: wait for
-          // the P V of step j - 1 (the one before it completed before S_x(j)).
-          const uint32_t pv = g - 1;
-          if (!wait_all(o_done + 2 * x + (pv & 1), (pv >> 1) & 1, abort, ctl, kSiteFwdSoftmax)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        // Rare after an item's first steps: some row of this warp moves its
+        // reference max (no exponential on the common path).
+        if (__any_sync(0xffffffffu, grow)) {
+          const float alpha = grow ? ex2(m - m_cand) : 1.f;
+          if (j > 0) {
+            // O_x must hold every earlier P V before it is rescaled: wait for
+            // the P V of step j - 1 (the one before it completed before S_x(j)).
+            const uint32_t pv = g - 1;
+            if (!wait_all(o_done + 2 * x + (pv & 1), (pv >> 1) & 1, abort, ctl, kSiteFwdSoftmax)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t o16[16];
-            tmem_ld16(lane_base + col_o + c * 16, o16);
-            tmem_wait_ld();
+            for (int c = 0; c < D / 16; ++c) {
+              uint32_t o16[16];
+              tmem_ld16(lane_base + col_o + c * 16, o16);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
-            tmem_st16(lane_base + col_o + c * 16, o16);
+              for (int e = 0; e < 16; ++e)
+                o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
+              tmem_st16(lane_base + col_o + c * 16, o16);
+            }
           }
-        }
-        if (grow) {
-          l *= alpha;
-          m = m_cand;
+          if (grow) {
+            l *= alpha;
+            m = m_cand;
+          }
         }
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
         const float2 sc2 = make_float2(scale_log2, scale_log2);

@@ -53,6 +53,11 @@ constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold; keeps P <= 2^8
 #define FA_FP8_POLY_EVERY 0  // one column pair in this many uses the FMA-pipe exp2 (0: none)
 #endif
 constexpr int kPolyMod = FA_FP8_POLY_EVERY > 0 ? FA_FP8_POLY_EVERY : 1;
+// P of a step leaves the softmax in kPParts equal parts of kPCols 32-bit
+// columns (4 E4M3 probabilities each), one barrier per part.
+constexpr int kPParts = 2;
+constexpr int kPCols = 32 / kPParts;
+static_assert(kPCols % 16 == 0 && kPCols % 8 == 0, "P parts");
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -63,7 +68,7 @@ struct Cfg {
   static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + NST * TILE;
   static constexpr int BAR_OFF = V_OFF + NST * TILE;
-  static constexpr int NBAR = 2 + 4 * NST + 6 + 4;
+  static constexpr int NBAR = 2 + 4 * NST + 4 + 2 * kPParts + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
   static constexpr int SMEM = MISC_OFF + 48 + 1024;    // + slack for 1 KB alignment
   static constexpr int KSTEPS = (D + 31) / 32;         // S MMA k-steps (32 E4M3 each)
@@ -187,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + C::NST;
   uint64_t* v_empty = v_full + C::NST;
   uint64_t* s_full = v_empty + C::NST;  // [2] per tile
-  uint64_t* p_full = s_full + 2;        // [2] per tile
-  uint64_t* o_done = p_full + 2;        // [2] per tile
+  uint64_t* p_full = s_full + 2;        // [2 tiles][kPParts parts of P]
+  uint64_t* o_done = p_full + 2 * kPParts;  // [2] per tile
   uint64_t* nxt_full = o_done + 2;      // [2] next-item responses
   uint64_t* nxt_empty = nxt_full + 2;   // [2]
   uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(s_full + x, 1);
-      mbar_init(p_full + x, kBM);
+      for (int q = 0; q < kPParts; ++q) mbar_init(p_full + kPParts * x + q, kBM);
       mbar_init(o_done + x, 1);
       mbar_init(nxt_full + x, 1);
       mbar_init(nxt_empty + x, 9);  // MMA warp + 8 softmax warps
@@ -353,14 +358,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    auto issue_pv = [&](int x, int r, bool first) {  // O_x (+)= P_x V, P_x from TMEM
+    // O_x (+)= P_x V over the keys of k-steps [K0, K1) (32 keys each), P_x
+    // from TMEM; the last part signals o_done.
+    auto issue_pv = [&](int x, int r, bool first, auto k0, auto k1) {
+      constexpr int K0 = decltype(k0)::value, K1 = decltype(k1)::value;
       if (leader) {
         const SDesc vd = v_desc + (r % C::NST) * C::TILE;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 32; ++kk)
+        for (int kk = K0; kk < K1; ++kk)
           mma_ts_e4m3(tmem + 256 + x * kBN, tmem + x * kBN + kk * 8, vd + kk * 32 * 128,
                       kIdescPV, (!first || kk > 0) ? 1u : 0u);
-        mma_commit(o_done + x);
+        if (K1 == kBN / 32) mma_commit(o_done + x);
       }
       __syncwarp();
     };
@@ -395,12 +403,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int x = 0; ok && x < 2; ++x) {
           if (j >= n_x[x]) continue;
-          if (!wait_all(p_full + x, (p_base[x] + j) & 1, abort, ctl, kSiteFp8Mma)) {
+          // P_x arrives in parts; each part's k-steps go as soon as it is in.
+          bool got = true;
+          static_for<kPParts>([&](auto q) {
+            constexpr int Q = decltype(q)::value;
+            if (!got) return;
+            got = wait_all(p_full + kPParts * x + Q, (p_base[x] + j) & 1, abort, ctl,
+                           kSiteFp8Mma);
+            if (!got) return;
+            tc_fence_after();
+            issue_pv(x, r, j == 0, std::integral_constant<int, Q * kPCols / 8>{},
+                     std::integral_constant<int, (Q + 1) * kPCols / 8>{});
+          });
+          if (!got) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          issue_pv(x, r, j == 0);
           if (j + 1 < n_x[x]) {
             if (!wait_k(r + 1)) {
               ok = false;
@@ -480,30 +498,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (c >= lim) s[c] = -INFINITY;
         }
-        float mx4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-        for (int c = 4; c < kBN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float mx = row_max(s);
         const float m_cand = fmaxf(m, mx * sl2);
         const bool grow = m_cand > m + kRescaleLog2;  // true on the first tile
-        const float alpha = grow ? ex2(m - m_cand) : 1.f;
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O_x += P_x(j-1) V completed before S_x(j) (same issuing thread,
-          // in order), so O_x can be rescaled now.
+        // Rare after an item's first steps: some row of this warp moves its
+        // reference max (no exponential on the common path).
+        if (__any_sync(0xffffffffu, grow)) {
+          const float alpha = grow ? ex2(m - m_cand) : 1.f;
+          if (j > 0) {
+            // O_x += P_x(j-1) V completed before S_x(j) (same issuing thread,
+            // in order), so O_x can be rescaled now.
 #pragma unroll
-          for (int c = 0; c < C::NPV / 16; ++c) {
-            uint32_t o16[16];
-            tmem_ld16(lane_base + col_o + c * 16, o16);
-            tmem_wait_ld();
+            for (int c = 0; c < C::NPV / 16; ++c) {
+              uint32_t o16[16];
+              tmem_ld16(lane_base + col_o + c * 16, o16);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
-            tmem_st16(lane_base + col_o + c * 16, o16);
+              for (int e = 0; e < 16; ++e)
+                o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
+              tmem_st16(lane_base + col_o + c * 16, o16);
+            }
           }
-        }
-        if (grow) {
-          l *= alpha;
-          m = m_cand;
+          if (grow) {
+            l *= alpha;
+            m = m_cand;
+          }
         }
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
         const float2 sc2 = make_float2(sl2, sl2);
@@ -511,8 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                          make_float2(0.f, 0.f)};
         uint32_t pk[kBN / 4];
-#pragma unroll
-        for (int c = 0; c < kBN / 4; ++c) {
+        // Four probabilities per 32-bit column (E4M3), 32 columns per row.
+        auto exp_quad = [&](int c) {
           float2 p2[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -532,13 +551,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             p2[h] = p;
           }
           pk[c] = pack_e4m3x4(p2[0].x, p2[0].y, p2[1].x, p2[1].y);
-        }
-        const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
-        l += rsa.x + rsa.y;
-        tmem_st32(lane_base + col_s, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full + x);
+        };
+        // P leaves in kPParts parts of kPCols columns, each with its own
+        // barrier, so the P V MMA starts on the first keys early.
+        static_for<kPParts>([&](auto q) {
+          constexpr int Q = decltype(q)::value;
+#pragma unroll
+          for (int c = Q * kPCols; c < (Q + 1) * kPCols; ++c) exp_quad(c);
+          if (Q == kPParts - 1) {
+            const float2 rsa =
+                __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+            l += rsa.x + rsa.y;
+          }
+#pragma unroll
+          for (int c = Q * kPCols; c < (Q + 1) * kPCols; c += 16)
+            tmem_st16(lane_base + col_s + c, *reinterpret_cast<const uint32_t(*)[16]>(&pk[c]));
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_full + kPParts * x + Q);
+        });
       }
       // -------------------------------------------------------- epilogue
       if (ok && wait_all(o_done + x, (s_base + n_kv - 1) & 1, abort, ctl, kSiteFp8Epilogue)) {

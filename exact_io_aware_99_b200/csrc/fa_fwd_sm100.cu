@@ -32,7 +32,11 @@
 //               per query row (= TMEM lane), base-2 domain, lazy rescaling
 //               (the reference max moves, and O and l are rescaled in TMEM,
 //               only when the row max grew by more than 2^8; exponents stay
-//               <= 8).  They also run their tile's epilogue (O / l, LSE):
+//               <= 8).  P leaves in two halves (keys 0-63, then 64-127),
+//               each with its own barrier, so the P V MMA starts on the first
+//               half while the second half is exponentiated (measured +1-2 %;
+//               four quarters cost more in barriers than they gain).  They
+//               also run their tile's epilogue (O / l, LSE):
 //               each warp writes its 32 rows of O, 64 columns at a time,
 //               into its own 4 KB swizzled staging buffer and one lane
 //               stores it with TMA (whole rows per transfer instead of one
@@ -74,6 +78,15 @@ constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 #define FA_FWD_POLY_EVERY 0  // one column pair in this many uses the FMA-pipe exp2 (0: none)
 #endif
 constexpr int kPolyMod = FA_FWD_POLY_EVERY > 0 ? FA_FWD_POLY_EVERY : 1;
+#ifndef FA_FWD_P_PARTS
+#define FA_FWD_P_PARTS 2
+#endif
+// P of a step leaves the softmax in kPParts equal parts (kPCols bf16 pairs,
+// i.e. 2 kPCols keys, each with its own barrier), so the P V MMA starts on
+// the first keys while the last exponentials are still being computed.
+constexpr int kPParts = FA_FWD_P_PARTS;
+constexpr int kPCols = kBN / 2 / kPParts;
+static_assert(kPParts >= 1 && kPCols % 16 == 0 && kPCols * kPParts == kBN / 2, "P parts");
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -88,7 +101,7 @@ struct Cfg {
   static constexpr int STG_OFF = V_OFF + NST * TILE;  // [8 softmax warps] 4 KB O staging
   static constexpr int STG = 4096;                     // 32 rows x 64 bf16 columns
   static constexpr int BAR_OFF = STG_OFF + 8 * STG;
-  static constexpr int NBAR = 2 + 4 * NST + 6 + 4;
+  static constexpr int NBAR = 2 + 4 * NST + 4 + 2 * kPParts + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
   static constexpr int SMEM = MISC_OFF + 48 + 1024;    // + slack for 1 KB alignment
   static constexpr int KSTEPS = D / 16;
@@ -232,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + C::NST;
   uint64_t* v_empty = v_full + C::NST;
   uint64_t* s_full = v_empty + C::NST;  // [2] per tile
-  uint64_t* p_full = s_full + 2;        // [2] per tile
-  uint64_t* o_done = p_full + 2;        // [2] per tile
+  uint64_t* p_full = s_full + 2;        // [2 tiles][kPParts parts of P]
+  uint64_t* o_done = p_full + 2 * kPParts;  // [2] per tile
   // Next-item requests (cluster launch control), double-buffered: the
   // producer issues the request for item i + 1 into slot (i + 1) & 1 once it
   // has issued item i's loads; the MMA warp and the 8 softmax warps read it
@@ -261,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(s_full + x, 1);
-      mbar_init(p_full + x, kBM);
+      for (int q = 0; q < kPParts; ++q) mbar_init(p_full + kPParts * x + q, kBM);
       mbar_init(o_done + x, 1);
       mbar_init(nxt_full + x, 1);
       mbar_init(nxt_empty + x, 9);  // MMA warp + 8 softmax warps
@@ -457,14 +470,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    auto issue_pv = [&](int x, int r, bool first) {  // O_x (+)= P_x V, P_x from TMEM
+    // O_x (+)= P_x V over the keys of k-steps [K0, K1) (16 keys each), P_x
+    // from TMEM; the last part signals o_done.
+    auto issue_pv = [&](int x, int r, bool first, auto k0, auto k1) {
+      constexpr int K0 = decltype(k0)::value, K1 = decltype(k1)::value;
       if (leader) {
         const SDesc vd = v_desc + (r % C::NST) * C::TILE;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
+        for (int kk = K0; kk < K1; ++kk)
           mma_ts(tmem + 256 + x * kBN, tmem + x * kBN + kk * 8, vd + kk * 16 * 128, kIdescPV,
                  (!first || kk > 0) ? 1u : 0u);
-        mma_commit(o_done + x);
+        if (K1 == kBN / 16) mma_commit(o_done + x);
       }
       __syncwarp();
     };
@@ -505,12 +521,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int x = 0; ok && x < 2; ++x) {
           if (j >= n_x[x]) continue;
-          if (!wait_all(p_full + x, (p_base[x] + j) & 1, abort, ctl, kSiteFwdMma)) {
+          // P_x arrives in parts; each part's k-steps go as soon as it is in.
+          bool got = true;
+          static_for<kPParts>([&](auto q) {
+            constexpr int Q = decltype(q)::value;
+            if (!got) return;
+            got = wait_all(p_full + kPParts * x + Q, (p_base[x] + j) & 1, abort, ctl,
+                           kSiteFwdMma);
+            if (!got) return;
+            tc_fence_after();
+            issue_pv(x, r, j == 0, std::integral_constant<int, Q * kPCols / 8>{},
+                     std::integral_constant<int, (Q + 1) * kPCols / 8>{});
+          });
+          if (!got) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          issue_pv(x, r, j == 0);
           if (j + 1 < n_x[x]) {
             if (!wait_k(r + 1)) {
               ok = false;
@@ -627,30 +653,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (c >= lim) s[c] = -INFINITY;
         }
-        float mx4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-        for (int c = 4; c < kBN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float mx = row_max(s);
         const float m_cand = fmaxf(m, mx * scale_log2);
         const bool grow = m_cand > m + kRescaleLog2;  // true on the first tile
-        const float alpha = grow ? ex2(m - m_cand) : 1.f;
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O_x += P_x(j-1) V completed before S_x(j) (same MMA thread, in
-          // order), so O_x can be rescaled now.
+        // Rare after an item's first steps: some row of this warp moves its
+        // reference max (no exponential on the common path).
+        if (__any_sync(0xffffffffu, grow)) {
+          const float alpha = grow ? ex2(m - m_cand) : 1.f;
+          if (j > 0) {
+            // O_x += P_x(j-1) V completed before S_x(j) (same MMA thread, in
+            // order), so O_x can be rescaled now.
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t o16[16];
-            tmem_ld16(lane_base + col_o + c * 16, o16);
-            tmem_wait_ld();
+            for (int c = 0; c < D / 16; ++c) {
+              uint32_t o16[16];
+              tmem_ld16(lane_base + col_o + c * 16, o16);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
-            tmem_st16(lane_base + col_o + c * 16, o16);
+              for (int e = 0; e < 16; ++e)
+                o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
+              tmem_st16(lane_base + col_o + c * 16, o16);
+            }
           }
-        }
-        if (grow) {
-          l *= alpha;
-          m = m_cand;
+          if (grow) {
+            l *= alpha;
+            m = m_cand;
+          }
         }
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
         const float2 sc2 = make_float2(scale_log2, scale_log2);
@@ -660,8 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                          make_float2(0.f, 0.f)};
         uint32_t pk[kBN / 2];
-#pragma unroll
-        for (int c = 0; c < kBN / 2; ++c) {
+        auto exp_pair = [&](int c) {
           const float2 xx = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
           float2 p;
           if (FA_FWD_POLY_EVERY > 0 && c % kPolyMod == kPolyMod - 1) {
@@ -675,19 +701,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           rs2[c & 3] = __fadd2_rn(rs2[c & 3], p);
           pk[c] = pack_bf16(p.x, p.y);
-        }
-        const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
-        const float rs = rsa.x + rsa.y;
-        l += rs;
-        {
-          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-          tmem_st32(lane_base + col_s + 0, lo);
-          tmem_st32(lane_base + col_s + 32, hi);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full + x);
+        };
+        // P as bf16 pairs in columns [c0, c1) of S's region (16 at a time),
+        // then the part's barrier.
+        auto store_p = [&](auto c0, auto c1, uint64_t* bar) {
+#pragma unroll
+          for (int c = decltype(c0)::value; c < decltype(c1)::value; c += 16)
+            tmem_st16(lane_base + col_s + c, *reinterpret_cast<const uint32_t(*)[16]>(&pk[c]));
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar);
+        };
+        static_for<kPParts>([&](auto q) {
+          constexpr int Q = decltype(q)::value;
+#pragma unroll
+          for (int c = Q * kPCols; c < (Q + 1) * kPCols; ++c) exp_pair(c);
+          if (Q == kPParts - 1) {
+            const float2 rsa =
+                __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+            l += rsa.x + rsa.y;
+          }
+          store_p(std::integral_constant<int, Q * kPCols>{},
+                  std::integral_constant<int, (Q + 1) * kPCols>{}, p_full + kPParts * x + Q);
+        });
       }
       // -------------------------------------------------------- epilogue
       // o_done completes once per P V of this tile; its last phase of this

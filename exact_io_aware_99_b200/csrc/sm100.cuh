@@ -8,6 +8,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -431,6 +432,45 @@ __device__ __forceinline__ void regs_decrease() {
 }
 
 // ------------------------------------------------------------ arithmetic
+
+// f(std::integral_constant<int, 0>{}), ..., f(std::integral_constant<int, N - 1>{}):
+// a loop whose index is a compile-time constant in the body.
+template <int N, int I = 0, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (I < N) {
+    f(std::integral_constant<int, I>{});
+    static_for<N, I + 1>(f);
+  }
+}
+
+// Largest of three values (one instruction on sm_100; like fmaxf, a NaN
+// input is ignored in favour of the others).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Largest of N values (N a multiple of 8): eight independent chains of
+// three-input maxima, so the reduction is N/2 instructions about N/16 deep.
+template <int N>
+__device__ __forceinline__ float row_max(const float (&s)[N]) {
+  static_assert(N % 8 == 0 && N >= 16, "row_max wants a multiple of 8, at least 16");
+  constexpr int kPairs = (N - 8) / 16;  // steps that fold two more values per chain
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = s[i];
+#pragma unroll
+  for (int k = 0; k < kPairs; ++k)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = fmax3(acc[i], s[8 + 16 * k + i], s[16 + 16 * k + i]);
+#pragma unroll
+  for (int c = 8 + 16 * kPairs; c < N; c += 8)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = fmaxf(acc[i], s[c + i]);
+  return fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]),
+               fmaxf(acc[6], acc[7]));
+}
 
 // 2^x on the special-function unit (approximate, flush-to-zero).
 __device__ __forceinline__ float ex2(float x) {
