@@ -245,7 +245,7 @@ struct KvCfg : Shape<D> {
   static constexpr int LSE_OFF = DO_OFF + NDO * S::TILE; // [NQ] x 512 B: the Q tile's LSE2
   static constexpr int DV_OFF = LSE_OFF + NQ * 512;      // [NDO] x 512 B: the dO tile's D
   static constexpr int BAR_OFF = DV_OFF + NDO * 512;
-  static constexpr int NBAR = 22;
+  static constexpr int NBAR = 24;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
   static constexpr int USED = MISC_OFF + 48;
   // Slack for aligning the dynamic shared memory to 1 KB, as far as the
@@ -297,12 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = bars + 11;
   uint64_t* dp_full = bars + 12;
   uint64_t* p_full = bars + 13;    // both softmax warpgroups wrote P^T
-  uint64_t* ds_full = bars + 14;   // both wrote dS^T
+  uint64_t* ds_full = bars + 14;   // both wrote dS^T, queries [0, 32) of each half
   uint64_t* kv_done = bars + 15;   // the item's last dK: accumulators final
   uint64_t* kv_empty = bars + 16;  // the item's S^T and dP^T MMAs are done with K_j, V_j
   uint64_t* nxt_full = bars + 17;  // [2] next-item requests
   uint64_t* nxt_empty = bars + 19; // [2]
   uint64_t* s_read = bars + 21;    // both softmax warpgroups have S^T in registers
+  uint64_t* ds_full2 = bars + 22;  // both wrote dS^T, queries [32, 64) of each half
   uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 36);
@@ -349,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(s_read, 8);
     mbar_init(p_full, 8);
     mbar_init(ds_full, 8);
+    mbar_init(ds_full2, 8);
     mbar_init(kv_done, 1);
     *abort = 0;
     fence_barrier_init();
@@ -564,22 +566,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(do_empty + sd);
         }
         __syncwarp();
-        if (!wait_all(ds_full, g & 1, abort, ctl, kSiteBwdMma)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         // dK += dS^T Q_i: dS^T k-step kk at column 64*(kk/4) + 8*(kk%4) of
-        // the dS^T half of B.
-        if (leader) {
+        // the dS^T half of B.  dS^T arrives in two parts (k-steps with
+        // kk%4 < 2, then the rest), and each part's MMAs go as soon as it is in.
 #pragma unroll
-          for (int kk = 0; kk < kT / 16; ++kk)
-            mma_ts(tmem + kKvColDK, tmem + kKvColDP + kKvOffDS + (kk >> 2) * 64 + (kk & 3) * 8,
-                   qm + kk * 2048, kIdescAcc,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(q_empty + sq);
+        for (int part = 0; part < 2; ++part) {
+          if (!wait_all(part ? ds_full2 : ds_full, g & 1, abort, ctl, kSiteBwdMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (leader) {
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+              for (int k2 = 0; k2 < 2; ++k2) {
+                const int kk = 4 * kh + 2 * part + k2;
+                mma_ts(tmem + kKvColDK,
+                       tmem + kKvColDP + kKvOffDS + (kk >> 2) * 64 + (kk & 3) * 8,
+                       qm + kk * 2048, kIdescAcc, (it > 0 || kk > 0) ? 1u : 0u);
+              }
+            if (part) mma_commit(q_empty + sq);
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        if (!ok) break;
         if (it + 1 < n_iter && !issue_dp(it + 1)) {
           ok = false;
           break;
@@ -671,7 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         warp_arrive(p_full);
         // dS^T = P^T o (dP^T - D), formed as P dP - P D on column pairs
-        // (two paired fp32 operations per pair).
+        // (two paired fp32 operations per pair).  Each 32-query part goes
+        // to the last 32 of this half's dP^T columns as soon as it is formed.
         uint32_t dsk[32];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -690,11 +702,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             dsk[c * 16 + e / 2] = pack_bf16(ra.x, ra.y);
             dsk[c * 16 + e / 2 + 1] = pack_bf16(rb.x, rb.y);
           }
+          tmem_st16(lane_base + col_dp + kKvOffDS + 16 * c,
+                    *reinterpret_cast<const uint32_t(*)[16]>(&dsk[16 * c]));
+          tmem_wait_st();
+          warp_arrive(c ? ds_full2 : ds_full);
         }
-        // dS^T -> the last 32 of this half's dP^T columns.
-        tmem_st32(lane_base + col_dp + kKvOffDS, dsk);
-        tmem_wait_st();
-        warp_arrive(ds_full);
       }
       if (!ok) break;
       // Epilogue: dV (unscaled) and dK (times scale), 16-column steps split
@@ -736,7 +748,7 @@ struct QCfg : Shape<D> {
   static constexpr int K_OFF = DO_OFF + S::TILE;      // [NK]
   static constexpr int V_OFF = K_OFF + NK * S::TILE;  // [NV]
   static constexpr int BAR_OFF = V_OFF + NV * S::TILE;
-  static constexpr int NBAR = (13 + 2 * NK + 2 * NV + 1) & ~1;  // even: keeps MISC 16-byte aligned
+  static constexpr int NBAR = (15 + 2 * NK + 2 * NV + 1) & ~1;  // even: keeps MISC 16-byte aligned
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // 16-byte aligned (next-item responses)
   static constexpr int SMEM = MISC_OFF + 48 + 1024;
   static_assert(MISC_OFF % 16 == 0, "next-item responses need 16-byte alignment");
@@ -774,8 +786,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = v_empty + C::NV;
   uint64_t* s_read = s_full + 1;        // both softmax warpgroups have S in registers
   uint64_t* dp_full = s_read + 1;       // [2] per dP buffer
-  uint64_t* ds_full = dp_full + 2;      // [2] per dP buffer
-  uint64_t* nxt_full = ds_full + 2;     // [2] next-item requests
+  uint64_t* ds_full = dp_full + 2;      // [2 dP buffers][2 parts: keys 0-31, 32-63 of each half]
+  uint64_t* nxt_full = ds_full + 4;     // [2] next-item requests
   uint64_t* nxt_empty = nxt_full + 2;   // [2]
   uint8_t* nxt_resp = smem + C::MISC_OFF;  // [2] x 16 bytes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 32);
@@ -817,7 +829,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(dp_full + b, 1);
-      mbar_init(ds_full + b, 8);    // one arrival per softmax warp
+      mbar_init(ds_full + 2 * b, 8);      // one arrival per softmax warp
+      mbar_init(ds_full + 2 * b + 1, 8);
       mbar_init(nxt_full + b, 1);
       mbar_init(nxt_empty + b, 9);  // MMA warp + 8 softmax warps
     }
@@ -1019,23 +1032,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        if (!wait_all(ds_full + (g & 1), (g >> 1) & 1, abort, ctl, kSiteBwdMma)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         // dQ += dS_jj K_jj: key k-step kk (16 keys) of dS at column
-        // 64*(kk/4) + 8*(kk%4) of the dP buffer.
-        if (leader) {
-          const SDesc km = k_mn + s * C::TILE;
+        // 64*(kk/4) + 8*(kk%4) of the dP buffer.  dS arrives in two parts
+        // (k-steps with kk%4 < 2, then the rest); each part's MMAs go as soon
+        // as it is in.
 #pragma unroll
-          for (int kk = 0; kk < kT / 16; ++kk)
-            mma_ts(tmem + kQColDQ, tmem + kQColDP + (g & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
-                   km + kk * 2048, kIdescDq,
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(k_empty + s);
+        for (int part = 0; part < 2; ++part) {
+          if (!wait_all(ds_full + 2 * (g & 1) + part, (g >> 1) & 1, abort, ctl, kSiteBwdMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (leader) {
+            const SDesc km = k_mn + s * C::TILE;
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+              for (int k2 = 0; k2 < 2; ++k2) {
+                const int kk = 4 * kh + 2 * part + k2;
+                mma_ts(tmem + kQColDQ,
+                       tmem + kQColDP + (g & 1) * kT + (kk >> 2) * 64 + (kk & 3) * 8,
+                       km + kk * 2048, kIdescDq, (jj > 0 || kk > 0) ? 1u : 0u);
+              }
+            if (part) mma_commit(k_empty + s);
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        if (!ok) break;
       }
       if (!ok) break;
       if (leader) mma_commit(dq_done);
@@ -1106,22 +1129,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + col_dp, dpv[0]);
         tmem_ld32(lane_base + col_dp + 32, dpv[1]);
         tmem_wait_ld();
-        // dS = P o (dP - D), formed as P dP - P D on column pairs.
+        // dS = P o (dP - D), formed as P dP - P D on column pairs, into the
+        // first 32 of this half's dP columns (already read) in two parts of
+        // 32 keys, each signalled as soon as it is stored.
         uint32_t dsk[32];
         const float2 nd2 = make_float2(-my_d, -my_d);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int c0 = 2 * c, c1 = 2 * c + 1;
-          const float2 pp = make_float2(p[c0], p[c1]);
-          const float2 r = __ffma2_rn(pp, make_float2(__uint_as_float(dpv[c0 >> 5][c0 & 31]),
-                                                      __uint_as_float(dpv[c1 >> 5][c1 & 31])),
-                                      __fmul2_rn(pp, nd2));
-          dsk[c] = pack_bf16(r.x, r.y);
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int c = 16 * part; c < 16 * part + 16; ++c) {
+            const int c0 = 2 * c, c1 = 2 * c + 1;
+            const float2 pp = make_float2(p[c0], p[c1]);
+            const float2 r = __ffma2_rn(pp, make_float2(__uint_as_float(dpv[c0 >> 5][c0 & 31]),
+                                                        __uint_as_float(dpv[c1 >> 5][c1 & 31])),
+                                        __fmul2_rn(pp, nd2));
+            dsk[c] = pack_bf16(r.x, r.y);
+          }
+          tmem_st16(lane_base + col_dp + 16 * part,
+                    *reinterpret_cast<const uint32_t(*)[16]>(&dsk[16 * part]));
+          tmem_wait_st();
+          warp_arrive(ds_full + 2 * (g & 1) + part);
         }
-        // dS -> the first 32 of this half's dP columns (already read).
-        tmem_st32(lane_base + col_dp, dsk);
-        tmem_wait_st();
-        warp_arrive(ds_full + (g & 1));
       }
       if (!ok) break;
       // dq_done completes once per item; the next item's first dQ MMA
