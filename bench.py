@@ -146,6 +146,16 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def window(self, t0: float, t1: float):
+        """Median and lowest SM clock and the throttle reasons seen between
+        two ``time.perf_counter()`` readings (NVML samples only)."""
+        rows = [r for r in self.rows if t0 <= r[0] <= t1]
+        if not rows:
+            return None
+        reasons = sorted({name for r in rows for bit, name in self.REASONS.items() if r[2] & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in rows),
+                "sm_mhz_min": min(r[1] for r in rows), "reasons": reasons, "samples": len(rows)}
+
     def stop(self):
         out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         if self.nvml is not None:
@@ -423,6 +433,7 @@ def run_ours(args, peaks, peak_kind):
 # fit in L2 get a 256 MB write before every timed pass.
 
 EXTRA_ITERS = 10
+EXTRA_GAP_S = 0.5  # idle before each extra entry (lets the power draw settle)
 
 
 def _timed_passes(passes, stream, iters, flush=None):
@@ -509,15 +520,28 @@ def run_extras(fa, dev, stream, peaks, gpu_index):
     flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
     clocks = ClockSampler(gpu_index, period_s=0.005)
     clocks.start()
+    windows = []  # (entry dict, t0, t1): the clock samples of each entry's timed passes
+
+    def entry(fn):
+        # A short idle gap first, so that one entry's power draw does not cap
+        # the clock of the next; each entry then carries its own clocks.
+        torch.cuda.synchronize()
+        time.sleep(EXTRA_GAP_S)
+        t0 = time.perf_counter()
+        out = fn()
+        windows.append((out, t0, time.perf_counter()))
+        return out
+
     configs = {}
     w = workloads.WORKLOADS["fwd_d64"]
-    configs["fwd_d64"] = _dense_entry(fa, dev, stream, w.B, w.H, w.N, w.d, w.causal, False,
-                                      workloads.make_inputs(w), peak, flush)
+    x = workloads.make_inputs(w)
+    configs["fwd_d64"] = entry(lambda: _dense_entry(fa, dev, stream, w.B, w.H, w.N, w.d,
+                                                    w.causal, False, x, peak, flush))
     for name in ("long_d128", "gpt3_d80"):
         w = workloads.WORKLOADS[name]
         x = _projected_inputs(w, dev) if w.projected else workloads.make_inputs(w)
-        configs[name] = _dense_entry(fa, dev, stream, w.B, w.H, w.N, w.d, w.causal, True, x,
-                                     peak)
+        configs[name] = entry(lambda: _dense_entry(fa, dev, stream, w.B, w.H, w.N, w.d,
+                                                   w.causal, True, x, peak))
         del x
     vs_n = []
     for causal in (True, False):
@@ -526,7 +550,8 @@ def run_extras(fa, dev, stream, peaks, gpu_index):
             B = max(1, 262144 // (H * N))
             x = {n: _device_randn((B, H, N, d), 5000 + 10 * N + i + 7 * causal, dev)
                  for i, n in enumerate(("q", "k", "v", "do"))}
-            vs_n.append(_dense_entry(fa, dev, stream, B, H, N, d, causal, True, x, peak))
+            vs_n.append(entry(lambda: _dense_entry(fa, dev, stream, B, H, N, d, causal, True, x,
+                                                   peak)))
             del x
     # FP8 forward at the target shape (E4M3 codes from the library's own
     # per-tensor quantiser), L2 flushed before every pass
@@ -540,7 +565,7 @@ def run_extras(fa, dev, stream, peaks, gpu_index):
     def f8():
         fa.fa_forward_fp8(q8, k8, v8, qd, kd, vd, o8, l8, w.B, w.H, w.N, w.d, w.scale, w.causal,
                           stream.cuda_stream)
-    ms8 = _timed_passes([f8], stream, EXTRA_ITERS, flush)[0]
+    ms8 = entry(lambda: {"ms": _timed_passes([f8], stream, EXTRA_ITERS, flush)[0]})["ms"]
     tf8 = perf.fwd_flops(w.B, w.H, w.N, w.d, w.causal) / (ms8 * 1e-3) / 1e12
     fp8 = {"workload": w.describe(), "fwd_ms": round(ms8, 4), "fwd_tflops": round(tf8, 2),
            "frac_of_fp8_peak": round(tf8 / (2 * peak), 4),
@@ -561,7 +586,7 @@ def run_extras(fa, dev, stream, peaks, gpu_index):
     def fdec():
         fa.fa_forward_splitkv(qd_, kd_, vd_, od_, ld_, w.B, w.H, w.N, w.nk, w.d, w.scale,
                               w.causal, splits, wsb, wb, stream.cuda_stream)
-    msd = _timed_passes([fdec], stream, EXTRA_ITERS)[0]
+    msd = entry(lambda: {"ms": _timed_passes([fdec], stream, EXTRA_ITERS)[0]})["ms"]
     nbytes = perf.decode_bytes(w.B, w.H, w.N, w.nk, w.d)
     gbs = nbytes / (msd * 1e-3) / 1e9
     decode = {"workload": w.describe(), "num_splits": splits, "fwd_ms": round(msd, 4),
@@ -571,14 +596,24 @@ def run_extras(fa, dev, stream, peaks, gpu_index):
               "algorithmic_bytes": nbytes,
               "l2": "K/V %.2f GB > 126 MB L2" % (2 * w.B * w.H * w.nk * w.d * 2 / 1e9)}
     clk = clocks.stop()
+    win = [clocks.window(t0, t1) for _, t0, t1 in windows]
+    for (out, _, _), c in zip(windows, win):
+        if c is not None:
+            out["clocks"] = c
+    # the FP8 and decode timings went through scratch dicts (the last two)
+    if win[-2] is not None:
+        fp8["clocks"] = win[-2]
+    if win[-1] is not None:
+        decode["clocks"] = win[-1]
     st, site = fa.fa_device_status(reset=True)
     if st != 0:
         raise RuntimeError(f"device wait timed out in the extra measurements (site {site:#x})")
     return {"configs": configs, "vs_n": vs_n, "fp8_fwd": fp8, "decode": decode,
             "extras_clocks": clk,
             "extras_note": "each entry CUDA-event timed in this process after 3 warm-up "
-                           f"steps, mean of {EXTRA_ITERS} timed passes; fractions of the "
-                           "measured bf16 peak (burst)"}
+                           f"steps, mean of {EXTRA_ITERS} timed passes, after {EXTRA_GAP_S} s "
+                           "idle; its 'clocks' are the NVML samples of its own timed passes; "
+                           "fractions of the measured bf16 peak (burst)"}
 
 
 # ------------------------------------------------------------- CPU oracle
