@@ -74,8 +74,11 @@ struct RegSplit {
   static_assert(2 * kSoftmax + kControl <= 3 * kLaunchRegs, "register split over budget");
 };
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
+// One column pair in FA_FWD_POLY_EVERY uses the FMA-pipe exp2 (0: none).
+// Measured on B200 with P in two halves: 1 in 8 +1.1 % (N = 4096 causal),
+// +1.9 % (N = 16384), +2.2 % (d = 80); 1 in 16 +1.1 / +1.3 %; 1 in 4 slower.
 #ifndef FA_FWD_POLY_EVERY
-#define FA_FWD_POLY_EVERY 0  // one column pair in this many uses the FMA-pipe exp2 (0: none)
+#define FA_FWD_POLY_EVERY 8
 #endif
 constexpr int kPolyMod = FA_FWD_POLY_EVERY > 0 ? FA_FWD_POLY_EVERY : 1;
 #ifndef FA_FWD_P_PARTS
