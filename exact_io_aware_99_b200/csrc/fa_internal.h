@@ -101,11 +101,11 @@ cudaError_t launch_fwd_splitkv_sm100(const CUtensorMap& tq, const CUtensorMap& t
 cudaError_t launch_splitkv_combine(const float* part_o, const float* part_lse, void* o,
                                    float* lse, int n_split, int rows, int d, const Launch& L);
 
-// Backward: the dQ kernel then the dK/dV kernel, in stream order.  The dQ
-// kernel computes the row statistics D = rowsum(dO o O) and LSE2 = LSE log2(e)
-// from o, dO (bf16 [BH, N, d]) and lse and writes them to dvec and lse2
+// Backward: the row-statistics kernel, the dQ kernel, then the dK/dV kernel,
+// in stream order.  The first computes D = rowsum(dO o O) and LSE2 =
+// LSE log2(e) from o, dO (bf16 [BH, N, d]) and lse into dvec and lse2
 // ([BH, Np] fp32, Np = N rounded up to 128; D = 0 and LSE2 = +inf past N),
-// where the dK/dV kernel reads them; dq, dk, dv are bf16 [BH, N, d] outputs.
+// which the other two read; dq, dk, dv are bf16 [BH, N, d] outputs.
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tdo, const void* o, const void* dO,
                              const float* lse, float* dvec, float* lse2, void* dq, void* dk,
