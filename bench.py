@@ -410,7 +410,7 @@ def run_ours(args, peaks, peak_kind):
         "frac_of_sustained_peak": round(value / ws / peak_s, 4),
         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json bf16_tflops burst {peak}, "
                        f"sustained {peak_s})",
-        "roofline": {"kernel": "fa_backward (dQ kernel + dK/dV kernel)",
+        "roofline": {"kernel": "fa_backward (row statistics + dQ kernel + dK/dV kernel)",
                      "bound": "tensor", "achieved": round(bwd_tf, 3), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(bwd_tf / peak, 4),
                      "traffic": traffic,
