@@ -37,6 +37,11 @@
 //    right behind it into the other buffer.  dQ is written once, in bf16, at
 //    the end: no atomics and no fp32 dQ buffer, at the price of recomputing
 //    S and dP (7 tile MMAs per tile pair instead of 5).
+//  In both kernels dS leaves the softmax in two parts (32 of each half's 64
+//  columns), each with its own barrier, so dK / dQ start on the first part;
+//  the accumulators leave through row stores split by column halves between
+//  the warpgroups, for d = 128 as whole 128-byte lines (an in-warp
+//  transpose, store_rows_t128).
 // Warp roles (both kernels, 10 warps): warps 0-3 and 4-7 are two softmax
 // warpgroups splitting the 128 columns of every tile in halves (one thread
 // per TMEM lane), warp 8 is the TMA producer, warp 9 the TMEM allocator and
