@@ -37,7 +37,7 @@ int forward_key_tile(int d, int N, int causal) {
   const int forced = g_fwd_key_tile.load(std::memory_order_relaxed);
   if (forced == 64 || forced == 128) return forced;
   if (!causal) return 128;
-  return N <= (d == 64 ? 512 : 256) ? 64 : 128;
+  return N <= (d == 128 ? 256 : 512) ? 64 : 128;
 }
 thread_local int g_last_cuda_error = 0;
 

@@ -268,6 +268,8 @@ def test_forward_key_tile_table_and_override():
     assert m.fa_forward_key_tile(128, 256, True) == 64
     assert m.fa_forward_key_tile(128, 257, True) == 128
     assert m.fa_forward_key_tile(80, 200, True) == 64
+    assert m.fa_forward_key_tile(80, 512, True) == 64
+    assert m.fa_forward_key_tile(80, 513, True) == 128
     assert m.fa_forward_key_tile(64, 512, True) == 64
     assert m.fa_forward_key_tile(64, 513, True) == 128
     assert m.fa_forward_key_tile(128, 128, False) == 128
