@@ -284,3 +284,12 @@ def test_forward_key_tile_table_and_override():
     finally:
         m.fa_set_forward_key_tile(0)
     assert m.fa_forward_key_tile(128, 16384, False) == 128
+
+
+def test_profile_source_hash_ignores_comments_only():
+    # a profile's recorded traffic stays valid across comment edits of the
+    # kernel sources, and not across code edits
+    import bench
+    code = "int a = 1; // one\n/* block\n comment */\nint b = a + 2;\n"
+    assert bench._code_only(code) == bench._code_only("int a = 1;\n\nint b = a + 2; // two\n")
+    assert bench._code_only(code) != bench._code_only("int a = 1;\nint b = a + 3;\n")
